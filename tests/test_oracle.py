@@ -1,0 +1,304 @@
+"""Pins for the CPU oracle, each against something other than the oracle itself.
+
+The pages print no worked numeric example, so the oracle is pinned by closed
+forms (dense softmax attention, direct block means), brute force on tiny
+inputs (top-K over explicit candidate sets), identities the method implies
+(a coarse token with weight B^l equals B^l identical fine tokens), central
+finite differences, and a hand-worked reordering table.  CPU only.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+# ----------------------------------------------------------------- sizes
+
+def test_level_sizes_match_the_workloads():
+    # [Trainable LLSA summary, §三]: level l holds N / B^l tokens; the finest
+    # list length is K unless fewer candidates exist.
+    p = oracle.Problem(H=256, W=256, d=64, B=16, L=4, K=8)
+    n, kl = p.levels()
+    assert n == [65536, 4096, 256, 16, 1]
+    assert kl == [0, 8, 8, 8, 1]
+    p = oracle.Problem(H=128, W=128, d=64, B=16, L=3, K=8)
+    assert p.levels() == ([16384, 1024, 64, 4], [0, 8, 8, 4])
+    p = oracle.Problem(H=32, W=32, d=64, B=16, L=2, K=4)
+    assert p.levels() == ([1024, 64, 4], [0, 4, 4])
+    p = oracle.Problem(H=512, W=512, d=64, B=16, L=4, K=8)
+    assert p.levels() == ([262144, 16384, 1024, 64, 4], [0, 8, 8, 8, 4])
+    with pytest.raises(ValueError):
+        oracle.Problem(H=40, W=32, d=8, B=16, L=2, K=4).levels()
+
+
+# --------------------------------------------------------------- reorder
+
+def test_reorder_matches_hand_worked_table():
+    want = np.loadtxt(os.path.join(GOLDEN, "reorder_8x8_B4_L2.txt"), dtype=np.int64)
+    p = oracle.Problem(H=8, W=8, d=1, B=4, L=2, K=1)
+    got = oracle.reorder_index(p).reshape(8, 8)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("H,W,B,L", [(32, 32, 16, 2), (16, 48, 16, 2), (64, 64, 16, 3), (24, 16, 4, 3)])
+def test_reorder_is_a_bijection_of_squares(H, W, B, L):
+    p = oracle.Problem(H=H, W=W, d=3, B=B, L=L, K=1)
+    h = oracle.reorder_index(p)
+    assert sorted(h.tolist()) == list(range(H * W))
+    t = int(round(B ** 0.5))
+    ys, xs = np.divmod(np.arange(H * W), W)
+    for l in range(1, L + 1):
+        # every aligned run of B^l hierarchical positions is one t^l x t^l square
+        run = h // (B ** l)
+        sq = (ys // t ** l) * (W // t ** l) + xs // t ** l
+        for r in np.unique(run):
+            assert len(np.unique(sq[run == r])) == 1
+    rng = np.random.default_rng(0)
+    x = _rand(rng, 2, H * W, 3)
+    xh = oracle.reorder(p, x, True)
+    np.testing.assert_array_equal(oracle.reorder(p, xh, False), x)
+    np.testing.assert_array_equal(xh[:, h, :], x)
+
+
+# ------------------------------------------------------------------ pool
+
+def test_pool_is_the_direct_block_mean():
+    # recursive mean over B tokens equals the direct mean over B^l tokens
+    rng = np.random.default_rng(1)
+    p = oracle.Problem(H=64, W=64, d=5, B=16, L=3, K=4)
+    x = _rand(rng, 3, p.N, p.d)
+    pyr = oracle.pool(p, x)
+    for l in range(1, p.L + 1):
+        want = x.reshape(3, p.N // 16 ** l, 16 ** l, p.d).mean(axis=2)
+        np.testing.assert_allclose(pyr[l - 1], want, rtol=1e-13, atol=1e-13)
+
+
+def test_pool_after_reorder_averages_pixel_squares():
+    rng = np.random.default_rng(2)
+    p = oracle.Problem(H=32, W=64, d=2, B=16, L=2, K=4)
+    img = _rand(rng, 1, p.H, p.W, p.d)
+    pyr = oracle.pool(p, oracle.reorder(p, img.reshape(1, p.N, p.d), True))
+    h = oracle.reorder_index(p).reshape(p.H, p.W)
+    for l in (1, 2):
+        s = 4 ** l
+        for Y in range(0, p.H, s):
+            for X in range(0, p.W, s):
+                j = h[Y, X] // 16 ** l
+                want = img[0, Y:Y + s, X:X + s].reshape(-1, p.d).mean(axis=0)
+                np.testing.assert_allclose(pyr[l - 1][0, j], want, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------- selection
+
+def _brute_select(p, pq, pk):
+    """Top-down brute force: full score matrices and explicit candidate masks."""
+    n, kl = p.levels()
+    out = [None] * p.L
+    for l in range(p.L, 0, -1):
+        BH = pq[l - 1].shape[0]
+        res = np.zeros((BH, n[l], kl[l]), np.int32)
+        for s in range(BH):
+            S = pq[l - 1][s] @ pk[l - 1][s].T
+            for a in range(n[l]):
+                if l == p.L:
+                    cand = np.arange(n[l])
+                else:
+                    parents = out[l][s, a // p.B]
+                    cand = np.array([c for c in range(n[l]) if (c // p.B) in set(parents.tolist())])
+                order = np.lexsort((cand, -S[a, cand]))
+                res[s, a] = np.sort(cand[order[: kl[l]]])
+        out[l - 1] = res
+    return out
+
+
+@pytest.mark.parametrize("H,W,B,L,K", [(32, 32, 16, 2, 4), (64, 64, 16, 3, 3), (16, 16, 4, 3, 2), (32, 32, 4, 3, 5)])
+def test_select_equals_brute_force(H, W, B, L, K):
+    rng = np.random.default_rng(H + L + K)
+    p = oracle.Problem(H=H, W=W, d=6, B=B, L=L, K=K)
+    x_q, x_k = _rand(rng, 2, p.N, p.d), _rand(rng, 2, p.N, p.d)
+    pq, pk = oracle.pool(p, x_q), oracle.pool(p, x_k)
+    got = oracle.select(p, pq, pk)
+    want = _brute_select(p, pq, pk)
+    for l in range(p.L):
+        np.testing.assert_array_equal(got[l], want[l])
+
+
+def test_select_children_lie_under_parent_picks():
+    p = oracle.Problem(H=128, W=128, d=16, B=16, L=3, K=8)
+    q, k, _ = synthetic.qkv(5, 1, 2, p.H, p.W, p.d, 4.0, bf16=False)
+    pq = oracle.pool(p, oracle.reorder(p, q, True))
+    pk = oracle.pool(p, oracle.reorder(p, k, True))
+    idx = oracle.select(p, pq, pk)
+    n, kl = p.levels()
+    for l in range(1, p.L):
+        child, parent = idx[l - 1], idx[l]
+        for s in range(child.shape[0]):
+            for a in range(n[l]):
+                assert set((child[s, a] // p.B).tolist()) <= set(parent[s, a // p.B].tolist())
+                assert np.all(np.diff(child[s, a]) > 0)
+
+
+def test_select_ties_keep_lower_index_and_k_all_keeps_everything():
+    p = oracle.Problem(H=64, W=64, d=4, B=16, L=2, K=3)
+    n, kl = p.levels()
+    pq = [np.ones((1, n[1], 4)), np.ones((1, n[2], 4))]
+    pk = [np.ones((1, n[1], 4)), np.ones((1, n[2], 4))]      # every score ties
+    idx = oracle.select(p, pq, pk)
+    assert (idx[1] == np.arange(3)).all()                     # lowest three coarse ids
+    assert (idx[0] == np.arange(3)).all()                     # children of coarse 0 only
+    pall = oracle.Problem(H=64, W=64, d=4, B=16, L=2, K=10 ** 6)
+    rng = np.random.default_rng(3)
+    pq = [_rand(rng, 1, n[1], 4), _rand(rng, 1, n[2], 4)]
+    pk = [_rand(rng, 1, n[1], 4), _rand(rng, 1, n[2], 4)]
+    idx = oracle.select(pall, pq, pk)
+    assert (idx[1] == np.arange(n[2])).all() and (idx[0] == np.arange(n[1])).all()
+
+
+def test_select_level_ranks_its_candidates():
+    rng = np.random.default_rng(4)
+    p = oracle.Problem(H=32, W=32, d=6, B=16, L=2, K=4)
+    pq, pk = oracle.pool(p, _rand(rng, 1, p.N, 6)), oracle.pool(p, _rand(rng, 1, p.N, 6))
+    idx = oracle.select(p, pq, pk)
+    got, rid, rsc = oracle.select_level(p, 1, pq, pk, idx, R=6)
+    np.testing.assert_array_equal(got, idx[0])
+    for a in range(got.shape[1]):
+        assert np.all(np.diff(rsc[0, a]) <= 0)
+        assert sorted(rid[0, a, :4].tolist()) == got[0, a].tolist()
+        np.testing.assert_allclose(rsc[0, a], [pq[0][0, a] @ pk[0][0, c] for c in rid[0, a]], rtol=1e-12)
+
+
+# ------------------------------------------------------------- attention
+
+def _dense(q, k, v, scale):
+    S = np.einsum("bnd,bmd->bnm", q, k) * scale
+    m = S.max(axis=-1, keepdims=True)
+    e = np.exp(S - m)
+    return np.einsum("bnm,bmd->bnd", e / e.sum(-1, keepdims=True), v), (m + np.log(e.sum(-1, keepdims=True)))[..., 0]
+
+
+def test_k_all_without_enrichment_is_dense_attention():
+    rng = np.random.default_rng(5)
+    p = oracle.Problem(H=32, W=32, d=16, B=16, L=2, K=10 ** 6, enrich_mask=0)
+    q, k, v = (_rand(rng, 2, p.N, p.d) for _ in range(3))
+    r = oracle.forward(p, q, k, v)
+    o, lse = _dense(q, k, v, p.scale)
+    np.testing.assert_allclose(r["o"], o, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(r["lse"], lse, rtol=1e-12)
+
+
+def test_dense_gradients_match_autograd():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(6)
+    p = oracle.Problem(H=16, W=16, d=8, B=16, L=2, K=10 ** 6, enrich_mask=0)
+    q, k, v, g = (_rand(rng, 1, p.N, p.d) for _ in range(4))
+    r = oracle.forward(p, q, k, v)
+    dq, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g)
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    out = torch.softmax(tq @ tk.transpose(-1, -2) * p.scale, dim=-1) @ tv
+    (out * torch.tensor(g)).sum().backward()
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_coarse_weight_equals_b_pow_l_copies():
+    # [Trainable LLSA summary, §四] / [write-up, §三]: a coarse token stands for
+    # B^l fine tokens and is weighted by B^l.  When K and V are constant on
+    # every level-2 square, each coarse token equals each of the tokens it
+    # averages, so LLSA must equal plain softmax attention over the fine keys
+    # plus all B^l members of every picked coarse token, listed explicitly.
+    rng = np.random.default_rng(7)
+    p = oracle.Problem(H=64, W=64, d=8, B=16, L=3, K=4, enrich_mask=0b011)
+    n, kl = p.levels()
+    tile = 16 ** 2
+    kc, vc = _rand(rng, 1, p.N // tile, p.d), _rand(rng, 1, p.N // tile, p.d)
+    k = np.repeat(kc, tile, axis=1)
+    v = np.repeat(vc, tile, axis=1)
+    q = _rand(rng, 1, p.N, p.d) * 2.0
+    r = oracle.forward(p, q, k, v)
+    idx = r["idx"]
+    for i in range(0, p.N, 37):
+        keys = [c * 16 + t for c in idx[0][0, i // 16] for t in range(16)]
+        for l in (1, 2):
+            for c in idx[l - 1][0, i // 16 ** l]:
+                keys += list(range(c * 16 ** l, (c + 1) * 16 ** l))
+        o, lse = _dense(q[:, i:i + 1], k[:, keys], v[:, keys], p.scale)
+        np.testing.assert_allclose(r["o"][0, i], o[0, 0], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(r["lse"][0, i], lse[0, 0], rtol=1e-12)
+
+
+def test_row_subset_equals_full_forward():
+    rng = np.random.default_rng(8)
+    p = oracle.Problem(H=32, W=32, d=8, B=16, L=2, K=4)
+    q, k, v = (_rand(rng, 1, p.N, p.d) for _ in range(3))
+    r = oracle.forward(p, q, k, v)
+    rows = np.array([0, 5, 100, 1023])
+    o, lse = oracle.attn_fwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], rows=rows)
+    np.testing.assert_array_equal(o[0, rows], r["o"][0, rows])
+    np.testing.assert_array_equal(lse[0, rows], r["lse"][0, rows])
+
+
+def _loss(p, q, k, v, idx, g):
+    pk, pv = oracle.pool(p, k), oracle.pool(p, v)
+    o, _ = oracle.attn_fwd(p, q, k, v, pk, pv, idx)
+    return float((o * g).sum())
+
+
+@pytest.mark.parametrize("d,K,mask,sample", [(8, 4, 0b11, None), (64, 4, 0b11, 40), (8, 16, 0b10, 400)])
+def test_backward_matches_finite_differences(d, K, mask, sample):
+    # N = 256 (16 x 16 pixels), B = 16, L = 2; index lists frozen; fp64
+    # central differences through pooling and attention.
+    rng = np.random.default_rng(9 + d + K)
+    p = oracle.Problem(H=16, W=16, d=d, B=16, L=2, K=K, enrich_mask=mask)
+    q, k, v, g = (_rand(rng, 1, p.N, d) for _ in range(4))
+    r = oracle.forward(p, q, k, v)
+    idx = r["idx"]
+    dq, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], idx, g)
+    h = 1e-6
+    for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+        flat = list(range(p.N * d))
+        if sample:
+            flat = rng.choice(p.N * d, size=sample, replace=False)
+        for e in flat:
+            t, c = divmod(int(e), d)
+            args = {"q": q, "k": k, "v": v}
+            plus = {n_: a.copy() for n_, a in args.items()}
+            minus = {n_: a.copy() for n_, a in args.items()}
+            plus[which][0, t, c] += h
+            minus[which][0, t, c] -= h
+            fd = (_loss(p, plus["q"], plus["k"], plus["v"], idx, g)
+                  - _loss(p, minus["q"], minus["k"], minus["v"], idx, g)) / (2 * h)
+            assert abs(fd - grad[0, t, c]) <= 1e-6 * max(1.0, abs(fd)), (which, t, c, fd, grad[0, t, c])
+
+
+# ------------------------------------------------------- index transpose
+
+@pytest.mark.parametrize("H,W,L,K", [(32, 32, 2, 4), (128, 128, 3, 8), (64, 64, 3, 10 ** 6)])
+def test_transpose_is_the_exact_inverse(H, W, L, K):
+    rng = np.random.default_rng(10)
+    p = oracle.Problem(H=H, W=W, d=4, B=16, L=L, K=K)
+    pq, pk = oracle.pool(p, _rand(rng, 2, p.N, 4)), oracle.pool(p, _rand(rng, 2, p.N, 4))
+    idx = oracle.select(p, pq, pk)
+    offs, ql = oracle.index_transpose(p, idx)
+    n, kl = p.levels()
+    for l in range(1, p.L + 1):
+        for s in range(2):
+            o, lst, ix = offs[l - 1][s], ql[l - 1][s], idx[l - 1][s]
+            assert o[0] == 0 and o[-1] == n[l] * kl[l] and np.all(np.diff(o) >= 0)
+            pairs_csr = {(int(a), int(j)) for a in range(n[l]) for j in ix[a]}
+            pairs_csc = set()
+            for j in range(n[l]):
+                seg = lst[o[j]:o[j + 1]]
+                assert np.all(np.diff(seg) > 0)
+                pairs_csc |= {(int(a), j) for a in seg}
+            assert pairs_csr == pairs_csc
+            assert len(pairs_csc) == n[l] * kl[l]
