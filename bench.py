@@ -1,0 +1,470 @@
+"""Benchmark: LLSA forward + backward tokens/s at 256 x 256 pixels (N = 65536).
+
+One step = one pass of the whole path over one batch: pool Q, K, V ->
+coarse-to-fine selection -> sparse attention forward -> index transpose ->
+sparse attention backward, through the C ABI of libllsa.so, on the 256^2
+workload (batch 2, 6 heads, d = 64, B = 16, L = 4, K = 8, bf16 tokens).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Every (batch, head) slice is independent, so N GPUs run N independent
+copies of the workload (one process per GPU, weak scaling, no data-path
+collective; the process group only carries the barrier and the max over
+ranks of the device time).  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (the plain fp64 restatement of the
+method, test infrastructure) on the host cores, on a bounded sample of the
+same workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="px256", batch=2, heads=6, H=256, W=256, d=64, B=16, L=4, K=8, sigma=4.0)
+METRIC = "LLSA fwd+bwd tokens/s at 256² pixels (N=65536); % of roofline"
+UNIT = "tokens/s"
+
+
+def config_desc(extra=None):
+    w = WORKLOAD
+    c = {"workload": f"{w['H']}x{w['W']} pixels, N={w['H'] * w['W']}, batch {w['batch']}, {w['heads']} heads, "
+                     f"d={w['d']}, B={w['B']}, L={w['L']}, K={w['K']}, enrichment at every level, bf16 tokens, "
+                     f"pool+select+attn_fwd+index_transpose+attn_bwd per step",
+         "tokens_per_step_per_gpu": w["batch"] * w["H"] * w["W"],
+         "inputs": f"seeded smooth fields (Gaussian sigma={w['sigma']} px, +0.1 white noise), dO ~ N(0,1)",
+         "l2": "no flush: inputs larger than L2 (Q, K, V, dO = 403 MB per step vs 126 MB L2)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = False
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
+        pg = True
+    return rank, local, world, pg
+
+
+def barrier(pg):
+    if pg:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    if not pg:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.ident = str(device_index)
+        try:
+            import torch
+            u = torch.cuda.get_device_properties(device_index).uuid
+            self.ident = "GPU-" + str(u)
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.ident, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------ roofline
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def algorithmic_bytes(stage: str, n, kl, BH: int, N: int, d: int, L: int) -> float:
+    """Compulsory HBM bytes of one call of a stage (every operand read once,
+    every result written once), bf16 tokens, fp32 pyramids / LSE, int32 lists."""
+    tok = BH * N * d * 2
+    pyr = BH * sum(n[l] for l in range(1, L + 1)) * d * 4
+    idx = BH * sum(n[l] * kl[l] for l in range(1, L + 1)) * 4
+    offs = BH * sum(n[l] + 1 for l in range(1, L + 1)) * 4
+    lse = BH * N * 4
+    if stage == "pool":          # per tensor: read x, write its pyramid
+        return tok + pyr
+    if stage == "select":        # read pooled Q and K of every level, write the lists
+        return 2 * pyr + idx
+    if stage == "attn_fwd":      # read Q, K, V, pooled K, V, lists; write O, LSE
+        return 3 * tok + 2 * pyr + idx + tok + lse
+    if stage == "index_transpose":   # read lists, write offsets + query lists
+        return idx + offs + idx
+    if stage == "attn_bwd":      # read Q, K, V, O, dO, LSE, pooled K, V, lists, CSC; write dQ, dK, dV
+        return 5 * tok + lse + 2 * pyr + idx + offs + idx + 3 * tok
+    raise ValueError(stage)
+
+
+def traffic_record(kernel_stage: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources are unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic_px256.txt")
+    if not os.path.exists(path):
+        return None
+    digest = sources_digest()
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 3 and f[0] == kernel_stage and not line.startswith("#"):
+            return float(f[1]) if f[2] == digest else None
+    return None
+
+
+def sources_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hierarchical_top_sparse_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------ our path
+
+STAGES = ("pool", "select", "attn_fwd", "index_transpose", "attn_bwd")
+
+
+def run_ours(args, rank, local, world, pg):
+    import numpy as np
+    import torch
+
+    import synthetic
+    from hierarchical_top_sparse_b200 import llsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    p = llsa.Problem(batch=w["batch"], heads=w["heads"], height=w["H"], width=w["W"], d=w["d"], B=w["B"],
+                     L=w["L"], K=w["K"], dtype=llsa.BF16)
+    seed = 1000 * rank
+    q, k, v = synthetic.qkv(seed, w["batch"], w["heads"], w["H"], w["W"], w["d"], w["sigma"])
+    g = synthetic.upstream_grad(seed + 1, w["batch"], w["heads"], p.N, w["d"])
+    host = [torch.from_numpy(x) for x in (q, k, v, g)]
+    raster = [h.to(dev).to(torch.bfloat16) for h in host]
+    # a DiT reorders once per network, not per attention call: untimed
+    hier = [torch.empty_like(x) for x in raster]
+    for src, dst in zip(raster, hier):
+        llsa.reorder(p, src, dst, True)
+    qd, kd, vd, gd = hier
+    del raster
+    pipe = llsa.Pipeline(p, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        llsa.pool(p, qd, pipe.pyrQ)
+        llsa.pool(p, kd, pipe.pyrK)
+        llsa.pool(p, vd, pipe.pyrV)
+        if ev is not None:
+            ev[1].record(stream)
+        llsa.select(p, pipe.pyrQ, pipe.pyrK, pipe.idx)
+        if ev is not None:
+            ev[2].record(stream)
+        llsa.attn_fwd(p, qd, kd, vd, pipe.pyrK, pipe.pyrV, pipe.idx, pipe.o, pipe.lse)
+        if ev is not None:
+            ev[3].record(stream)
+        llsa.index_transpose(p, pipe.idx, pipe.offs, pipe.qlist, pipe.tscratch)
+        if ev is not None:
+            ev[4].record(stream)
+        llsa.attn_bwd(p, qd, kd, vd, pipe.o, gd, pipe.lse, pipe.pyrK, pipe.pyrV, pipe.idx, pipe.offs, pipe.qlist,
+                      pipe.dq, pipe.dk, pipe.dv, pipe.work)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if llsa.device_error() != 0:
+        raise RuntimeError("a bounded device wait gave up during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    barrier(pg)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = llsa.kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = llsa.kernel_launches() - launches0
+    barrier(pg)
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(ms_total, pg, dev)
+    ms_step = ms_total / args.steps
+    tokens_step = w["batch"] * p.N
+    value = world * tokens_step * args.steps / (ms_total / 1e3)
+
+    stage_ms = {}
+    for j, name in enumerate(STAGES):
+        stage_ms[name] = sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)) / args.steps
+
+    # roofline of the dominant kernel call, and of every stage
+    n, kl = llsa.level_sizes(p)
+    peak, peak_kind = peaks()
+    stages = {}
+    for name in STAGES:
+        calls = 3 if name == "pool" else 1
+        b = algorithmic_bytes(name, n, kl, p.BH, p.N, p.d, p.L) * calls
+        gbs = b / (stage_ms[name] / 1e3) / 1e9
+        stages[name] = {"ms": round(stage_ms[name], 4), "algorithmic_MB": round(b / 1e6, 2),
+                        "achieved_GBs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    dom = max(STAGES, key=lambda s: stage_ms[s])
+    traffic = traffic_record(dom)
+    roof = {"bound": "hbm", "kernel": dom, "achieved": stages[dom]["achieved_GBs"], "peak": peak,
+            "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else
+            "fallback 6650 GB/s", "unit": "GB/s", "frac": stages[dom]["frac"],
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": stages[dom]["algorithmic_MB"] * 1e6 / (3 if dom == "pool" else 1)}
+    # whole-step fraction: all compulsory bytes at HBM bandwidth vs the measured step
+    step_bytes = sum(algorithmic_bytes(s, n, kl, p.BH, p.N, p.d, p.L) * (3 if s == "pool" else 1) for s in STAGES)
+    step_floor_ms = step_bytes / (peak * 1e9) * 1e3
+
+    # end to end through host buffers: H2D of Q, K, V, dO (pinned), the path,
+    # D2H of O, LSE, dQ, dK, dV
+    e2e = None
+    if not args.no_e2e:
+        pinned_in = [llsa_pin(torch, hier_host) for hier_host in (qd, kd, vd, gd)]
+        outs = (pipe.o, pipe.lse, pipe.dq, pipe.dk, pipe.dv)
+        pinned_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in pinned_in)
+        d2h = sum(t.numel() * t.element_size() for t in pinned_out)
+        e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            for src, dst in zip(pinned_in, (qd, kd, vd, gd)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for src, dst in zip(outs, pinned_out):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(pg)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier(pg)
+        e_ms = max_over_ranks(a0.elapsed_time(a1), pg, dev)
+        e2e = {"value": round(world * tokens_step * e_steps / (e_ms / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e_steps,
+               "ms_per_step": round(e_ms / e_steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_desc({"parallelism": f"{world} independent replicas (batch x heads slices), "
+                                                      "no collective"}),
+                "roofline": roof,
+                "step_roofline": {"bound": "hbm", "compulsory_MB": round(step_bytes / 1e6, 1),
+                                  "floor_ms": round(step_floor_ms, 4), "frac": round(step_floor_ms / ms_step, 4)},
+                "stages": stages, "gpu_launches": launches, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+
+
+def llsa_pin(torch, t):
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
+
+
+# ---------------------------------------------------------- the oracle arm
+
+def oracle_sample_step(op, inputs, rows, slices):
+    """One bounded sample of the workload on the CPU oracle: the whole path
+    (pool, select, forward, transpose, backward) of ``slices`` (batch, head)
+    slices, with the attention forward and backward run for ``rows`` query
+    rows of each slice.  Returns the number of query tokens processed."""
+    import oracle
+    qh, kh, vh, gh = inputs
+    sel = slice(0, slices)
+    pq, pk, pv = oracle.pool(op, qh[sel]), oracle.pool(op, kh[sel]), oracle.pool(op, vh[sel])
+    idx = oracle.select(op, pq, pk)
+    oracle.attn_fwd(op, qh[sel], kh[sel], vh[sel], pk, pv, idx, rows=rows)
+    oracle.index_transpose(op, idx)
+    oracle.attn_bwd(op, qh[sel], kh[sel], vh[sel], pk, pv, idx, gh[sel], rows=rows)
+    return slices * len(rows)
+
+
+def oracle_setup():
+    import numpy as np
+
+    import oracle
+    import synthetic
+    w = WORKLOAD
+    op = oracle.Problem(H=w["H"], W=w["W"], d=w["d"], B=w["B"], L=w["L"], K=w["K"])
+    q, k, v = synthetic.qkv(0, w["batch"], w["heads"], w["H"], w["W"], w["d"], w["sigma"])
+    g = synthetic.upstream_grad(1, w["batch"], w["heads"], op.N, w["d"])
+    BH = w["batch"] * w["heads"]
+    slices = min(BH, os.cpu_count() or 1)
+    inputs = [oracle.reorder(op, x.reshape(BH, op.N, w["d"])[:slices], True) for x in (q, k, v, g)]
+    return op, inputs, slices
+
+
+def cpu_baseline(budget_s: float = 20.0):
+    import numpy as np
+    op, inputs, slices = oracle_setup()
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(op.N, size=2048, replace=False))
+    t = time.perf_counter()
+    tokens = oracle_sample_step(op, inputs, rows, slices)
+    dt = time.perf_counter() - t
+    reps = 1
+    while time.perf_counter() - t + dt < budget_s and reps < 8:
+        tokens += oracle_sample_step(op, inputs, rows, slices)
+        reps += 1
+    dt = time.perf_counter() - t
+    return {"value": round(tokens / dt, 1), "unit": UNIT, "cores": min(slices, os.cpu_count() or 1),
+            "kind": "oracle",
+            "sample": f"{reps} x (pool+select+transpose of {slices} (batch,head) slices of the 256^2 workload, "
+                      f"attention fwd+bwd for {len(rows)} sampled query rows of each; fp64 C oracle, one thread "
+                      f"per slice); tokens = query rows attended"}
+
+
+def run_reference(args, rank, world, pg):
+    if rank != 0:
+        barrier(pg)
+        return
+    import numpy as np
+    op, inputs, slices = oracle_setup()
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(op.N, size=256, replace=False))
+    for _ in range(args.warmup):
+        oracle_sample_step(op, inputs, rows, slices)
+    t = time.perf_counter()
+    tokens = 0
+    for _ in range(args.steps):
+        tokens += oracle_sample_step(op, inputs, rows, slices)
+    dt = time.perf_counter() - t
+    value = tokens / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_desc({"parallelism": "CPU oracle on the host cores (rank 0 only)"}),
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": slices, "kind": "oracle",
+                             "sample": f"per step: pool+select+transpose of {slices} (batch,head) slices of the "
+                                       f"256^2 workload, attention fwd+bwd for {len(rows)} sampled query rows "
+                                       f"of each; tokens = query rows attended"},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    barrier(pg)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank, local, world, pg = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world, pg)
+        else:
+            run_ours(args, rank, local, world, pg)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,90 @@
+// llsa_internal.cuh -- shared definitions of the CUDA side (never seen by callers).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "llsa.h"
+
+namespace llsa {
+
+// Derived sizes of one problem, computed on the host and passed to kernels by value.
+struct Geo {
+  int BH;          // batch * heads
+  int H, W;        // image size
+  int N;           // tokens per slice
+  int d;           // head dimension
+  int B;           // block size
+  int t;           // sqrt(B)
+  int L;           // levels
+  int K;           // requested top-K
+  unsigned emask;  // enriched levels, bit l-1 = level l
+  float scale;     // softmax scale
+  int bf16;        // 1: bf16 tensors, 0: fp32
+  int n[LLSA_MAX_LEVELS + 1];        // tokens per level (n[0] = N)
+  int Kl[LLSA_MAX_LEVELS + 1];       // list length per level (Kl[0] = 0)
+  int64_t Bl[LLSA_MAX_LEVELS + 1];   // B^l
+  int64_t pyr_off[LLSA_MAX_LEVELS + 2];   // element offset of level l in a pyramid (index L+1 = total)
+  int64_t idx_off[LLSA_MAX_LEVELS + 2];   // element offset of level l in idx / qlist
+  int64_t offs_off[LLSA_MAX_LEVELS + 2];  // element offset of level l in offs
+  int64_t cur_off[LLSA_MAX_LEVELS + 2];   // element offset of level l in the transpose cursors
+};
+
+// Fills g from p; returns LLSA_OK or the validation error.
+llsa_status make_geo(const llsa_problem* p, Geo* g);
+
+// Counts kernel launches issued by this library (host side, process wide).
+void note_launches(int n);
+
+// Device address of the error word that bounded waits set when they give up
+// (nullptr if the symbol cannot be resolved on the current device).
+int* device_error_word();
+
+// ----------------------------------------------------------------- launchers
+// All return cudaSuccess or the launch error; they assume a validated Geo.
+cudaError_t launch_reorder(const Geo& g, const void* in, void* out, int to_hier, cudaStream_t s);
+cudaError_t launch_pool(const Geo& g, const void* x, float* pyr, cudaStream_t s);
+cudaError_t launch_select_level(const Geo& g, int level, const float* pyrQ, const float* pyrK, int32_t* idx,
+                                cudaStream_t s);
+cudaError_t launch_index_transpose(const Geo& g, const int32_t* idx, int32_t* offs, int32_t* qlist,
+                                   int32_t* cursor, cudaStream_t s);
+cudaError_t launch_attn_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
+                            const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
+cudaError_t launch_attn_bwd(const Geo& g, const void* q, const void* k, const void* v, const void* o,
+                            const void* dO, const float* lse, const float* pyrK, const float* pyrV,
+                            const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
+                            void* dv, void* workspace, cudaStream_t s);
+
+// CUDA-core (fp32 FMA) attention kernels.
+cudaError_t launch_attn_fwd_simt(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
+                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
+cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, const void* v, const void* o,
+                                 const void* dO, const float* lse, const float* pyrK, const float* pyrV,
+                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
+                                 void* dv, void* workspace, cudaStream_t s);
+
+// Largest candidate count the selection kernel keeps in shared memory.
+constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
+
+// Workspace of the backward pass: D [BH][N] fp32, then the fp32 level gradients
+// of the pooled K and of the pooled V (each a pyramid).
+inline size_t bwd_workspace_bytes(const Geo& g) {
+  size_t dsz = (size_t)g.BH * g.N * sizeof(float);
+  dsz = (dsz + 255) & ~(size_t)255;
+  size_t pyr = (size_t)g.pyr_off[g.L + 1] * sizeof(float);
+  pyr = (pyr + 255) & ~(size_t)255;
+  return dsz + 2 * pyr;
+}
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+}  // namespace llsa

@@ -21,6 +21,7 @@ Pinning status of every routine (the tests in ``tests/test_oracle.py``):
   select                    pinned: brute-force top-K, child invariant, ties, K = all
   attn_fwd                  pinned: dense softmax attention at K = all; B^l copies identity
   attn_bwd                  pinned: central finite differences; dense autograd at K = all
+  attn_dq_rows              pinned: equals the rows of attn_bwd's dQ
   index_transpose           pinned: exact inverse of the query-major lists
 """
 from __future__ import annotations
@@ -74,7 +75,9 @@ def _load():
         lib.oracle_select.argtypes = [P, vp, vp, vp]
         lib.oracle_attn_fwd_rows.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp]
         lib.oracle_attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.oracle_attn_bwd_rows.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp, vp]
         lib.oracle_index_transpose.argtypes = [P, vp, vp, vp]
+        lib.oracle_attn_dq_rows.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp]
         _lib = lib
     return _lib
 
@@ -247,9 +250,10 @@ def attn_fwd(p: Problem, q, k, v, pyrK, pyrV, idx, rows: Optional[np.ndarray] = 
     return o, lse
 
 
-def attn_bwd(p: Problem, q, k, v, pyrK, pyrV, idx, dO):
+def attn_bwd(p: Problem, q, k, v, pyrK, pyrV, idx, dO, rows: Optional[np.ndarray] = None):
     """(dQ, dK, dV, dPK, dPV): token gradients [BH, N, d] and the pooled-level
-    gradients (lists over l = 1..L) before they are sent back to the tokens."""
+    gradients (lists over l = 1..L) before they are sent back to the tokens.
+    With ``rows`` given only those queries contribute (a timing sample)."""
     n, _ = p.levels()
     qs, ks, vs, gs = (_as_slices(a, 2) for a in (q, k, v, dO))
     BH = qs.shape[0]
@@ -259,14 +263,17 @@ def attn_bwd(p: Problem, q, k, v, pyrK, pyrV, idx, dO):
     dpv = np.empty((BH, tot))
     cp = p.c()
 
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+
     def run(s):
         pk = _pack(pyrK, s, np.float64)
         pv = _pack(pyrV, s, np.float64)
         ix = _pack(idx, s, np.int32)
-        _load().oracle_attn_bwd(ctypes.byref(cp), qs[s].ctypes.data, ks[s].ctypes.data, vs[s].ctypes.data,
-                                pk.ctypes.data, pv.ctypes.data, ix.ctypes.data, gs[s].ctypes.data,
-                                dq[s].ctypes.data, dk[s].ctypes.data, dv[s].ctypes.data,
-                                dpk[s].ctypes.data, dpv[s].ctypes.data)
+        _load().oracle_attn_bwd_rows(ctypes.byref(cp), qs[s].ctypes.data, ks[s].ctypes.data, vs[s].ctypes.data,
+                                     pk.ctypes.data, pv.ctypes.data, ix.ctypes.data, gs[s].ctypes.data,
+                                     None if r is None else r.ctypes.data, 0 if r is None else len(r),
+                                     dq[s].ctypes.data, dk[s].ctypes.data, dv[s].ctypes.data,
+                                     dpk[s].ctypes.data, dpv[s].ctypes.data)
 
     _map(run, BH)
     lk, lv, o = [], [], 0
@@ -275,6 +282,26 @@ def attn_bwd(p: Problem, q, k, v, pyrK, pyrV, idx, dO):
         lv.append(dpv[:, o:o + n[l] * p.d].reshape(BH, n[l], p.d))
         o += n[l] * p.d
     return dq, dk, dv, lk, lv
+
+
+def attn_dq_rows(p: Problem, q, k, v, pyrK, pyrV, idx, dO, rows: np.ndarray):
+    """dQ [BH, N, d] for the listed query rows only (others NaN)."""
+    qs, ks, vs, gs = (_as_slices(a, 2) for a in (q, k, v, dO))
+    BH = qs.shape[0]
+    dq = np.full_like(qs, np.nan)
+    cp = p.c()
+    r = np.ascontiguousarray(rows, dtype=np.int64)
+
+    def run(s):
+        pk = _pack(pyrK, s, np.float64)
+        pv = _pack(pyrV, s, np.float64)
+        ix = _pack(idx, s, np.int32)
+        _load().oracle_attn_dq_rows(ctypes.byref(cp), qs[s].ctypes.data, ks[s].ctypes.data, vs[s].ctypes.data,
+                                    pk.ctypes.data, pv.ctypes.data, ix.ctypes.data, gs[s].ctypes.data,
+                                    r.ctypes.data, len(r), dq[s].ctypes.data)
+
+    _map(run, BH)
+    return dq
 
 
 def index_transpose(p: Problem, idx: Sequence[np.ndarray]):

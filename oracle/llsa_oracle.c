@@ -336,10 +336,13 @@ void oracle_attn_fwd(const oracle_problem* p, const double* q, const double* k, 
  * back to the B^l tokens it averages: dk_t += dPK_l[floor(t/B^l)] / B^l
  * (the same for v).  Pooled Q is used only for selection, so it receives
  * no gradient.  If dpk/dpv are not NULL they receive the pooled-level
- * gradients (same packing as a pyramid). */
-void oracle_attn_bwd(const oracle_problem* p, const double* q, const double* k, const double* v,
-                     const double* pyrK, const double* pyrV, const int32_t* idx, const double* dO,
-                     double* dq, double* dk, double* dv, double* dpk, double* dpv) {
+ * gradients (same packing as a pyramid).  With rows != NULL only the listed
+ * fine queries contribute (a bounded sample of the work, used to time the
+ * oracle); rows == NULL is the complete backward. */
+void oracle_attn_bwd_rows(const oracle_problem* p, const double* q, const double* k, const double* v,
+                          const double* pyrK, const double* pyrV, const int32_t* idx, const double* dO,
+                          const int64_t* rows, int64_t nrows, double* dq, double* dk, double* dv, double* dpk,
+                          double* dpv) {
   int64_t n[64], Kl[64];
   if (oracle_levels(p, n, Kl)) return;
   const int d = p->d;
@@ -357,7 +360,9 @@ void oracle_attn_bwd(const oracle_problem* p, const double* q, const double* k, 
   int* level = (int*)malloc(sizeof(int) * mk);
   int64_t* id = (int64_t*)malloc(sizeof(int64_t) * mk);
   double* o = (double*)malloc(sizeof(double) * d);
-  for (int64_t i = 0; i < n[0]; ++i) {
+  int64_t count = rows ? nrows : n[0];
+  for (int64_t r = 0; r < count; ++r) {
+    int64_t i = rows ? rows[r] : r;
     int64_t m = key_set(p, n, Kl, i, k, v, pyrK, pyrV, idx, kp, vp, bias, level, id);
     double zmax = -INFINITY;
     for (int64_t j = 0; j < m; ++j) {
@@ -414,6 +419,13 @@ void oracle_attn_bwd(const oracle_problem* p, const double* q, const double* k, 
   free(gpk); free(gpv); free(kp); free(vp); free(bias); free(z); free(level); free(id); free(o);
 }
 
+/* The whole backward: every fine query contributes. */
+void oracle_attn_bwd(const oracle_problem* p, const double* q, const double* k, const double* v,
+                     const double* pyrK, const double* pyrV, const int32_t* idx, const double* dO,
+                     double* dq, double* dk, double* dv, double* dpk, double* dpv) {
+  oracle_attn_bwd_rows(p, q, k, v, pyrK, pyrV, idx, dO, NULL, 0, dq, dk, dv, dpk, dpv);
+}
+
 /* ------------------------------------------------------ index transpose */
 
 /* Sparse index transpose, query-major lists to key-major lists ([ART] §四;
@@ -450,4 +462,53 @@ void oracle_index_transpose(const oracle_problem* p, const int32_t* idx, int32_t
     free(fill);
     off_base += n[l] + 1;
   }
+}
+
+/* dq for the fine queries listed in rows[0..nrows) only (the same formula as
+ * oracle_attn_bwd: dq_i = scale * sum_j P_ij (dO_i . v_j - D_i) k_j); each row
+ * needs nothing but its own key set, so it can be computed one by one. */
+void oracle_attn_dq_rows(const oracle_problem* p, const double* q, const double* k, const double* v,
+                         const double* pyrK, const double* pyrV, const int32_t* idx, const double* dO,
+                         const int64_t* rows, int64_t nrows, double* dq) {
+  int64_t n[64], Kl[64];
+  if (oracle_levels(p, n, Kl)) return;
+  const int d = p->d;
+  int64_t mk = max_keys(p, Kl);
+  const double** kp = (const double**)malloc(sizeof(double*) * mk);
+  const double** vp = (const double**)malloc(sizeof(double*) * mk);
+  double* bias = (double*)malloc(sizeof(double) * mk);
+  double* z = (double*)malloc(sizeof(double) * mk);
+  int* level = (int*)malloc(sizeof(int) * mk);
+  int64_t* id = (int64_t*)malloc(sizeof(int64_t) * mk);
+  double* o = (double*)malloc(sizeof(double) * d);
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t i = rows[r];
+    int64_t m = key_set(p, n, Kl, i, k, v, pyrK, pyrV, idx, kp, vp, bias, level, id);
+    double zmax = -INFINITY;
+    for (int64_t j = 0; j < m; ++j) {
+      double s = 0.0;
+      for (int e = 0; e < d; ++e) s += q[i * d + e] * kp[j][e];
+      z[j] = p->scale * s + bias[j];
+      if (z[j] > zmax) zmax = z[j];
+    }
+    double sum = 0.0;
+    for (int64_t j = 0; j < m; ++j) sum += exp(z[j] - zmax);
+    double lse = zmax + log(sum);
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    for (int64_t j = 0; j < m; ++j) {
+      double P = exp(z[j] - lse);
+      for (int e = 0; e < d; ++e) o[e] += P * vp[j][e];
+    }
+    double D = 0.0;
+    for (int e = 0; e < d; ++e) D += dO[i * d + e] * o[e];
+    for (int e = 0; e < d; ++e) dq[i * d + e] = 0.0;
+    for (int64_t j = 0; j < m; ++j) {
+      double P = exp(z[j] - lse);
+      double dP = 0.0;
+      for (int e = 0; e < d; ++e) dP += dO[i * d + e] * vp[j][e];
+      double dz = P * (dP - D);
+      for (int e = 0; e < d; ++e) dq[i * d + e] += p->scale * dz * kp[j][e];
+    }
+  }
+  free(kp); free(vp); free(bias); free(z); free(level); free(id); free(o);
 }

@@ -8,8 +8,8 @@ Recipe (stands in for the FFHQ / ImageNet pixel tokens the method is trained
 on; the datasets themselves are not used):
   * every (batch, head, channel) of Q, K and V is an independent H x W field
     of N(0, 1) noise,
-  * blurred by a separable Gaussian of width ``sigma`` pixels, truncated at
-    4 sigma, reflecting at the border,
+  * blurred by a Gaussian of width ``sigma`` pixels (periodic boundary,
+    applied as its exact transfer function in the Fourier domain),
   * standardised to zero mean and unit variance,
   * plus ``noise`` * N(0, 1) white noise,
   * laid out in raster order as [batch, heads, H*W, d];
@@ -17,16 +17,22 @@ on; the datasets themselves are not used):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
-from scipy.ndimage import gaussian_filter1d
+import scipy.fft
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even); returns float32."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    x = np.array(x, dtype=np.float32, copy=True, order="C")
+    u = x.view(np.uint32)              # finite values: no uint32 overflow below
+    lsb = (u >> 16) & 1
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u &= np.uint32(0xFFFF0000)
+    return x
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -35,30 +41,46 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     return (x.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def smooth_fields(rng: np.random.Generator, count: int, H: int, W: int, sigma: float,
-                  noise: float = 0.1) -> np.ndarray:
-    """``count`` independent smooth H x W fields as float32 [count, H, W]."""
+def _gaussian_transfer(H: int, W: int, sigma: float) -> np.ndarray:
+    fy = np.fft.fftfreq(H)[:, None]
+    fx = np.fft.rfftfreq(W)[None, :]
+    return np.exp(-2.0 * np.pi ** 2 * sigma ** 2 * (fy ** 2 + fx ** 2)).astype(np.float32)
+
+
+def smooth_fields(seed: int, count: int, H: int, W: int, sigma: float, noise: float = 0.1) -> np.ndarray:
+    """``count`` independent smooth H x W fields as float32 [count, H, W].
+
+    Fields are drawn in chunks, each from its own child stream of ``seed``
+    (numpy SeedSequence.spawn), so the result does not depend on the number
+    of threads that draw them."""
     out = np.empty((count, H, W), dtype=np.float32)
-    chunk = max(1, (1 << 24) // (H * W))
-    for s in range(0, count, chunk):
+    chunk = max(1, (1 << 21) // (H * W))
+    starts = list(range(0, count, chunk))
+    children = np.random.SeedSequence(seed).spawn(len(starts))
+    tf = _gaussian_transfer(H, W, sigma) if sigma > 0 else None
+
+    def one(i):
+        s = starts[i]
         e = min(count, s + chunk)
+        rng = np.random.default_rng(children[i])
         f = rng.standard_normal((e - s, H, W), dtype=np.float32)
-        if sigma > 0:
-            f = gaussian_filter1d(f, sigma, axis=1, mode="reflect", truncate=4.0)
-            f = gaussian_filter1d(f, sigma, axis=2, mode="reflect", truncate=4.0)
+        if tf is not None:
+            f = scipy.fft.irfft2(scipy.fft.rfft2(f) * tf, s=(H, W)).astype(np.float32)
         mu = f.mean(axis=(1, 2), keepdims=True)
         sd = f.std(axis=(1, 2), keepdims=True)
         f = (f - mu) / np.maximum(sd, 1e-12)
-        f = f + noise * rng.standard_normal((e - s, H, W), dtype=np.float32)
+        f += noise * rng.standard_normal((e - s, H, W), dtype=np.float32)
         out[s:e] = f
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(one, range(len(starts))))
     return out
 
 
 def pixel_tokens(seed: int, batch: int, heads: int, H: int, W: int, d: int, sigma: float,
                  noise: float = 0.1, bf16: bool = True) -> np.ndarray:
     """One [batch, heads, H*W, d] raster-order token tensor of smooth fields."""
-    rng = np.random.default_rng(seed)
-    f = smooth_fields(rng, batch * heads * d, H, W, sigma, noise)
+    f = smooth_fields(seed, batch * heads * d, H, W, sigma, noise)
     t = f.reshape(batch, heads, d, H * W).transpose(0, 1, 3, 2)
     t = np.ascontiguousarray(t)
     return round_to_bf16(t) if bf16 else t
@@ -74,8 +96,20 @@ def qkv(seed: int, batch: int, heads: int, H: int, W: int, d: int, sigma: float,
 
 def upstream_grad(seed: int, batch: int, heads: int, N: int, d: int, bf16: bool = True) -> np.ndarray:
     """dO ~ N(0, 1), [batch, heads, N, d]."""
-    rng = np.random.default_rng(seed)
-    g = rng.standard_normal((batch, heads, N, d), dtype=np.float32)
+    rows = batch * heads * N
+    g = np.empty((rows, d), dtype=np.float32)
+    chunk = max(1, (1 << 21) // d)
+    starts = list(range(0, rows, chunk))
+    children = np.random.SeedSequence(seed).spawn(len(starts))
+
+    def one(i):
+        s = starts[i]
+        e = min(rows, s + chunk)
+        g[s:e] = np.random.default_rng(children[i]).standard_normal((e - s, d), dtype=np.float32)
+
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(one, range(len(starts))))
+    g = g.reshape(batch, heads, N, d)
     return round_to_bf16(g) if bf16 else g
 
 

@@ -1,0 +1,206 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+* reorder, pyramids: exact / fp32 rounding only;
+* index lists: bit-exact per level with the oracle fed the GPU's parent lists,
+  except near-ties (K-th and (K+1)-th oracle scores within 1e-4 relative);
+* CSC lists: bit-exact against the oracle's transpose of the GPU's lists;
+* O, LSE, dQ, dK, dV: relative Frobenius <= 1e-2 and max-abs <= 2e-2 for bf16
+  (1e-4 for fp32), with the oracle fed the GPU's index lists, and end to end on
+  every row whose lists the oracle selected identically.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synthetic
+from parity_util import Case, GpuRun, assert_close, check_level_picks, errors, to_dev, to_np
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from hierarchical_top_sparse_b200 import llsa
+    llsa.lib()
+
+
+def check_selection(run: GpuRun):
+    """Level by level, coarsest first, the oracle fed the GPU's parent lists."""
+    op = run.op
+    n, kl = op.levels()
+    pq, pk = oracle.pool(op, run.qh), oracle.pool(op, run.kh)
+    ties = 0
+    for l in range(op.L, 0, -1):
+        want, rid, rsc = oracle.select_level(op, l, pq, pk, run.idx, R=kl[l] + 4)
+        got = run.idx[l - 1]
+        assert got.shape == want.shape
+        assert np.all(np.diff(got, axis=-1) > 0), f"level {l}: lists not strictly ascending"
+        if kl[l] < rsc.shape[-1]:
+            ties += check_level_picks(got, want, rid, rsc, kl[l])
+        else:
+            np.testing.assert_array_equal(got, want)
+    return ties
+
+
+def check_pyramids(run: GpuRun):
+    op = run.op
+    for name, src, got in (("Q", run.qh, run.pyrQ), ("K", run.kh, run.pyrK), ("V", run.vh, run.pyrV)):
+        want = oracle.pool(op, src)
+        for l in range(op.L):
+            np.testing.assert_allclose(got[l], want[l], rtol=2e-6, atol=2e-6, err_msg=f"pyramid {name} level {l + 1}")
+
+
+def check_transpose(run: GpuRun):
+    offs, ql = oracle.index_transpose(run.op, run.idx)
+    for l in range(run.op.L):
+        np.testing.assert_array_equal(run.offs[l], offs[l], err_msg=f"offsets level {l + 1}")
+        np.testing.assert_array_equal(run.qlist[l], ql[l], err_msg=f"query lists level {l + 1}")
+
+
+def check_attention(run: GpuRun, backward: bool, sel=slice(None)):
+    """Teacher-forced: the oracle attends with the GPU's index lists."""
+    op, dt = run.op, run.case.dtype
+    idx = [a[sel] for a in run.idx]
+    pk, pv = oracle.pool(op, run.kh[sel]), oracle.pool(op, run.vh[sel])
+    o, lse = oracle.attn_fwd(op, run.qh[sel], run.kh[sel], run.vh[sel], pk, pv, idx)
+    res = {"o": assert_close("O", run.o[sel], o, dt), "lse": assert_close("LSE", run.lse[sel], lse, dt)}
+    if backward:
+        dq, dk, dv, _, _ = oracle.attn_bwd(op, run.qh[sel], run.kh[sel], run.vh[sel], pk, pv, idx, run.gh[sel])
+        res["dq"] = assert_close("dQ", run.dq[sel], dq, dt)
+        res["dk"] = assert_close("dK", run.dk[sel], dk, dt)
+        res["dv"] = assert_close("dV", run.dv[sel], dv, dt)
+    return res
+
+
+def check_end_to_end(run: GpuRun, sel=slice(None), min_match=0.99):
+    """The oracle's own selection; rows whose lists all agree must agree in O."""
+    op, dt = run.op, run.case.dtype
+    r = oracle.forward(op, run.qh[sel], run.kh[sel], run.vh[sel])
+    n, _ = op.levels()
+    BH = r["o"].shape[0]
+    same = np.ones((BH, n[0]), bool)
+    for l in range(1, op.L + 1):
+        eq = np.all(r["idx"][l - 1] == run.idx[l - 1][sel], axis=-1)          # [BH, n_l]
+        same &= np.repeat(eq, op.B ** l, axis=1)
+    frac = same.mean()
+    assert frac >= min_match, f"only {frac:.4f} of the rows have identical index lists"
+    assert_close("O (end to end)", run.o[sel][same], r["o"][same], dt)
+    return frac
+
+
+CASES = {
+    # the smallest workload: 32 x 32 pixels, fp32, B = 16, L = 2, K = 4
+    "tiny32_fp32": Case(batch=1, heads=1, H=32, W=32, L=2, K=4, dtype="fp32"),
+    "px64_bf16": Case(batch=2, heads=2, H=64, W=64, L=3, K=8),
+    "px64_fp32_E2": Case(batch=1, heads=2, H=64, W=64, L=3, K=8, dtype="fp32", enrich_mask=0b010),
+    "px64_noenrich": Case(batch=1, heads=2, H=64, W=64, L=2, K=6, enrich_mask=0),
+    "single_level": Case(batch=1, heads=2, H=64, W=64, L=1, K=8),
+    "B4": Case(batch=1, heads=2, H=32, W=32, B=4, L=3, K=6, dtype="fp32"),
+    "B64": Case(batch=1, heads=2, H=64, W=64, B=64, L=2, K=3, d=32),
+    "d128_ragged_K": Case(batch=1, heads=1, H=64, W=48, L=2, K=5, d=128),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_small_cases_full_parity(name):
+    case = CASES[name]
+    run = GpuRun(case)
+    check_pyramids(run)
+    check_selection(run)
+    check_transpose(run)
+    check_attention(run, backward=True)
+    check_end_to_end(run, min_match=0.98)
+
+
+def test_reorder_roundtrip_is_exact():
+    case = Case(batch=1, heads=3, H=64, W=32, L=2)
+    from hierarchical_top_sparse_b200 import llsa
+    p, op = case.problems()
+    q, _, _, _ = case.inputs()
+    x = to_dev(q, True)
+    y = torch.empty_like(x)
+    z = torch.empty_like(x)
+    llsa.reorder(p, x, y, True)
+    llsa.reorder(p, y, z, False)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(y), oracle.reorder(op, q, True).astype(np.float32))
+    assert torch.equal(x, z)
+    p32 = llsa.Problem(batch=1, heads=3, height=64, width=32, L=2, dtype=llsa.FP32)
+    x32 = torch.from_numpy(q).cuda()
+    y32 = torch.empty_like(x32)
+    llsa.reorder(p32, x32, y32, True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y32.cpu().numpy(), oracle.reorder(op, q, True).astype(np.float32))
+
+
+def test_dense_when_k_covers_everything():
+    # K >= every candidate count and no enrichment: plain softmax attention
+    case = Case(batch=1, heads=1, H=32, W=32, L=2, K=10 ** 6, dtype="fp32", enrich_mask=0)
+    run = GpuRun(case)
+    q, k, v = run.qh[0], run.kh[0], run.vh[0]
+    S = (q.astype(np.float64) @ k.T.astype(np.float64)) * run.p.scale
+    P = np.exp(S - S.max(1, keepdims=True))
+    o = (P / P.sum(1, keepdims=True)) @ v
+    assert_close("O dense", run.o[0], o, "fp32")
+    check_attention(run, backward=True)
+    check_transpose(run)
+
+
+def test_select_and_transpose_are_deterministic():
+    case = Case(batch=2, heads=2, H=64, W=64, L=3, K=8)
+    a, b = GpuRun(case), GpuRun(case)
+    for l in range(3):
+        np.testing.assert_array_equal(a.idx[l], b.idx[l])
+        np.testing.assert_array_equal(a.qlist[l], b.qlist[l])
+
+
+@pytest.mark.parametrize("cfg", ["px128", "px128_fwd"])
+def test_workload_128(cfg):
+    c = synthetic.CONFIGS[cfg]
+    case = Case(batch=c["batch"], heads=c["heads"], H=c["H"], W=c["W"], L=c["L"], K=c["K"], sigma=c["sigma"])
+    run = GpuRun(case, backward=c["backward"])
+    check_pyramids(run)
+    ties = check_selection(run)
+    if c["backward"]:
+        check_transpose(run)
+    check_attention(run, backward=c["backward"])
+    check_end_to_end(run)
+    print(f"{cfg}: {ties} near-tie rows")
+
+
+def sampled_rows(N, count, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(N, size=count, replace=False))
+
+
+@pytest.mark.parametrize("cfg,full_slices", [("px256", (0, 7)), ("px512", ())])
+def test_workload_full_size(cfg, full_slices):
+    """The full-size workloads in the launch configuration the benchmark times:
+    every selection level and the transposes in full, O / LSE / dQ on sampled
+    rows of every slice, dK / dV of whole slices where the oracle finishes in
+    seconds, and the gradient-sum identities everywhere."""
+    c = synthetic.CONFIGS[cfg]
+    case = Case(batch=c["batch"], heads=c["heads"], H=c["H"], W=c["W"], L=c["L"], K=c["K"], sigma=c["sigma"])
+    run = GpuRun(case, backward=True)
+    op = run.op
+    check_selection(run)
+    check_transpose(run)
+    rows = sampled_rows(op.N, 512, 3)
+    pk, pv = oracle.pool(op, run.kh), oracle.pool(op, run.vh)
+    o, lse = oracle.attn_fwd(op, run.qh, run.kh, run.vh, pk, pv, run.idx, rows=rows)
+    assert_close("O rows", run.o[:, rows], o[:, rows], "bf16")
+    assert_close("LSE rows", run.lse[:, rows], lse[:, rows], "bf16")
+    dq = oracle.attn_dq_rows(op, run.qh, run.kh, run.vh, pk, pv, run.idx, run.gh, rows)
+    assert_close("dQ rows", run.dq[:, rows], dq[:, rows], "bf16")
+    # sum_t dV_t = sum_i dO_i and sum_t dK_t = 0, per slice and channel
+    sv = run.dv.astype(np.float64).sum(axis=1)
+    np.testing.assert_allclose(sv, run.gh.astype(np.float64).sum(axis=1), rtol=0, atol=0.5 + 2e-3 * np.abs(sv).max())
+    sk = run.dk.astype(np.float64).sum(axis=1)
+    scale_k = np.abs(run.dk).sum(axis=1)
+    assert np.all(np.abs(sk) <= 2e-2 * scale_k + 1e-3), "sum of dK is not ~0"
+    for s in full_slices:
+        check_attention(run, backward=True, sel=slice(s, s + 1))

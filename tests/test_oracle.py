@@ -302,3 +302,27 @@ def test_transpose_is_the_exact_inverse(H, W, L, K):
                 pairs_csc |= {(int(a), j) for a in seg}
             assert pairs_csr == pairs_csc
             assert len(pairs_csc) == n[l] * kl[l]
+
+
+def test_dq_rows_equal_full_backward_rows():
+    rng = np.random.default_rng(11)
+    p = oracle.Problem(H=32, W=32, d=8, B=16, L=2, K=4)
+    q, k, v, g = (_rand(rng, 2, p.N, p.d) for _ in range(4))
+    r = oracle.forward(p, q, k, v)
+    dq, _, _, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g)
+    rows = np.array([3, 64, 999])
+    got = oracle.attn_dq_rows(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g, rows)
+    np.testing.assert_allclose(got[:, rows], dq[:, rows], rtol=1e-13, atol=1e-14)
+
+
+def test_gradient_sums_hold():
+    # sum_t dV_t = sum_i dO_i (every softmax row sums to one) and sum_t dK_t = 0
+    # (sum_j P_ij (dO_i.v_j - D_i) = 0): properties used at sizes the oracle
+    # cannot finish.
+    rng = np.random.default_rng(12)
+    p = oracle.Problem(H=32, W=32, d=8, B=16, L=2, K=4)
+    q, k, v, g = (_rand(rng, 1, p.N, p.d) for _ in range(4))
+    r = oracle.forward(p, q, k, v)
+    _, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g)
+    np.testing.assert_allclose(dv.sum(axis=1), g.sum(axis=1), rtol=1e-12, atol=1e-11)
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-11)
