@@ -9,6 +9,8 @@
 // The scatter order is arbitrary, so a last pass writes each key's ids in
 // ascending order (short ranges by an in-register rank, long ranges through a
 // shared-memory bitmap of the query ids).
+#include <mutex>
+
 #include "llsa_internal.cuh"
 
 namespace llsa {
@@ -218,3 +220,61 @@ cudaError_t launch_index_transpose(const Geo& g, const int32_t* idx, int32_t* of
 }
 
 }  // namespace llsa
+
+// ----------------------------------------------- transpose without scratch
+//
+// llsa_index_transpose_noalloc: the same four kernels, with their scratch in a
+// fixed device array owned by this library instead of a caller buffer.  The
+// array is a file-scope __device__ object, so every GPU that loads the library
+// holds kNoAllocScratchBytes of it until the process exits.  Host code cannot
+// use the symbol's name as a device address: its address is looked up once
+// per device with cudaGetSymbolAddress (on the first call made while that
+// device is current) and cached.
+
+namespace llsa {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.
+static llsa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LLSA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return LLSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LLSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LLSA_OK;
+}
+
+}  // namespace llsa
+
+extern "C" llsa_status llsa_index_transpose_noalloc(const llsa_problem* p, const int32_t* idx, int32_t* offs,
+                                                    int32_t* qlist, llsa_stream stream) {
+  llsa::Geo g;
+  llsa_status st = llsa::make_geo(p, &g);
+  if (st != LLSA_OK) return st;
+  const void* bufs[3] = {idx, offs, qlist};
+  for (const void* b : bufs) {
+    if (!b) return LLSA_ERR_ARG;
+    if ((uintptr_t)b & 15u) return LLSA_ERR_ALIGN;
+  }
+  const size_t cur = ((size_t)g.cur_off[g.L + 1] * sizeof(int32_t) + 255) & ~(size_t)255;
+  const size_t need = cur + (size_t)g.idx_off[g.L + 1] * sizeof(int32_t);
+  if (need > llsa::kNoAllocScratchBytes) return LLSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = llsa::noalloc_scratch(&scratch);
+  if (st != LLSA_OK) return st;
+  cudaError_t e = llsa::launch_index_transpose(g, idx, offs, qlist, (int32_t*)scratch, (cudaStream_t)stream);
+  if (e != cudaSuccess || cudaPeekAtLastError() != cudaSuccess) return LLSA_ERR_CUDA;
+  return LLSA_OK;
+}

@@ -35,7 +35,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "alignment", 4: "worksp
 
 EXPORTS = ("llsa_status_string", "llsa_validate", "llsa_level_sizes", "llsa_query_sizes", "llsa_reorder",
            "llsa_pool", "llsa_select", "llsa_select_level", "llsa_attn_fwd", "llsa_index_transpose",
-           "llsa_attn_bwd", "llsa_device_error", "llsa_kernel_launches")
+           "llsa_attn_bwd", "llsa_device_error", "llsa_kernel_launches", "llsa_index_transpose_noalloc")
 
 
 class LLSAError(RuntimeError):
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "llsa_select_level": ([P, i32, vp, vp, vp, vp], i32),
             "llsa_attn_fwd": ([P, vp, vp, vp, vp, vp, vp, vp, vp, vp], i32),
             "llsa_index_transpose": ([P, vp, vp, vp, vp, vp], i32),
+            "llsa_index_transpose_noalloc": ([P, vp, vp, vp, vp], i32),
             "llsa_attn_bwd": ([P] + [vp] * 16, i32),
             "llsa_device_error": ([vp, ctypes.POINTER(i32)], i32),
             "llsa_kernel_launches": ([], ctypes.c_uint64),
@@ -199,6 +200,14 @@ def attn_fwd(p: Problem, q, k, v, pyrK, pyrV, idx, o, lse, stream=None):
 def index_transpose(p: Problem, idx, offs, qlist, scratch, stream=None):
     _check(lib().llsa_index_transpose(ctypes.byref(p.c()), _ptr(idx), _ptr(offs), _ptr(qlist), _ptr(scratch),
                                       _stream(stream)), "index_transpose")
+
+
+def index_transpose_noalloc(p: Problem, idx, offs, qlist, stream=None):
+    """index_transpose with the library's own fixed scratch array: for callers
+    that cannot allocate device memory.  Calls whose GPU work overlaps share
+    that array and must be serialized."""
+    _check(lib().llsa_index_transpose_noalloc(ctypes.byref(p.c()), _ptr(idx), _ptr(offs), _ptr(qlist),
+                                              _stream(stream)), "index_transpose_noalloc")
 
 
 def attn_bwd(p: Problem, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, dq, dk, dv, workspace, stream=None):

@@ -147,6 +147,28 @@ llsa_status llsa_attn_fwd(const llsa_problem* p, const void* q, const void* k, c
 llsa_status llsa_index_transpose(const llsa_problem* p, const int32_t* idx, int32_t* offs, int32_t* qlist,
                                  void* scratch, llsa_stream stream);
 
+/* llsa_index_transpose without a scratch argument.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot obtain
+ * device memory at the point where they run the transpose -- for example a
+ * plug-in whose host framework owns every device allocation and exposes no
+ * allocator to it, or a latency-critical loop that must never call
+ * cudaMalloc (which can synchronize the device).  Those callers still pass
+ * idx, offs and qlist, but no scratch: the scratch lives in a fixed 16 MiB
+ * device array inside this library (every GPU that loads the library holds
+ * it until the process exits).  A problem whose transpose needs more than
+ * that (transpose_scratch_bytes > 16 MiB) is rejected with
+ * LLSA_ERR_WORKSPACE before anything is launched.  Nothing is allocated:
+ * no cudaMalloc, no cudaFree.
+ * The first call on a device, made while that device is current, looks up
+ * the array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture.  All calls share the one array and it
+ * keeps whatever the last call left there (the parts that must start at zero
+ * are cleared by every call), so two calls whose work overlaps on the GPU --
+ * on different streams, or from different threads -- race and must be
+ * serialized by the caller.  Results are identical to llsa_index_transpose. */
+llsa_status llsa_index_transpose_noalloc(const llsa_problem* p, const int32_t* idx, int32_t* offs,
+                                         int32_t* qlist, llsa_stream stream);
+
 /* Sparse attention backward ([LLSA] §4.1), index lists held fixed.  With
  * P = exp(z - lse) and D_i = dO_i . o_i:  dq_i = scale * sum_j P_ij (dO_i.v_j - D_i) k_j;
  * fine keys gather their queries through the level-1 CSC lists (offs, qlist);
