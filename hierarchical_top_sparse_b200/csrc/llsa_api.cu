@@ -85,9 +85,12 @@ llsa_status make_geo(const llsa_problem* p, Geo* g) {
   return LLSA_OK;
 }
 
-// Attention dispatch: every problem currently runs on the CUDA-core kernels.
+// Attention dispatch: bf16 problems with d = 64 and B = 16 run on the tensor
+// cores; every other problem (fp32, other block sizes or head dims, K so large
+// that a group's picks or pooled keys overflow the tiles) on the CUDA cores.
 cudaError_t launch_attn_fwd(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                             const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s) {
+  if (attn_fwd_mma_supported(g)) return launch_attn_fwd_mma(g, q, k, v, pyrK, pyrV, idx, o, lse, s);
   return launch_attn_fwd_simt(g, q, k, v, pyrK, pyrV, idx, o, lse, s);
 }
 

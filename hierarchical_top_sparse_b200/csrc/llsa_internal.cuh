@@ -1,6 +1,7 @@
 // llsa_internal.cuh -- shared definitions of the CUDA side (never seen by callers).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -63,6 +64,15 @@ cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, con
                                  const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                  const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                  void* dv, void* workspace, cudaStream_t s);
+
+// Tensor-core attention kernels (bf16, d = 64, B = 16).
+bool attn_fwd_mma_supported(const Geo& g);
+cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
+                                const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
+
+// TMA descriptor of a [rows][64] bf16 token tensor, boxes of 16 rows x 64
+// columns (one 2 KB key or query block), 128-byte swizzle.
+cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows);
 
 // Largest candidate count the selection kernel keeps in shared memory.
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp

@@ -102,6 +102,9 @@ CASES = {
     "B4": Case(batch=1, heads=2, H=32, W=32, B=4, L=3, K=6, dtype="fp32"),
     "B64": Case(batch=1, heads=2, H=64, W=64, B=64, L=2, K=3, d=32),
     "d128_ragged_K": Case(batch=1, heads=1, H=64, W=48, L=2, K=5, d=128),
+    # tensor-core forward: level 1 not enriched; K = 16 (unions larger than the slot ring)
+    "px64_E23": Case(batch=2, heads=1, H=64, W=64, L=3, K=8, enrich_mask=0b110),
+    "px64_K16": Case(batch=1, heads=2, H=64, W=64, L=3, K=16),
 }
 
 
