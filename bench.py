@@ -89,13 +89,19 @@ def max_over_ranks(x: float, pg, device) -> float:
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 50 ms, timestamped) read on a thread; the
+    samples that fall inside the timed region (plus 100 ms either side) are
+    reported.  start() returns once the first sample has arrived."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device_index: int):
         self.proc = None
+        self.lines = []
+        self.thread = None
+        self.t_begin = self.t_end = None
         self.ident = str(device_index)
         try:
             import torch
@@ -104,41 +110,71 @@ class ClockSampler:
         except Exception:
             pass
 
+    def _reader(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", self.ident, f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
         except Exception:
             self.proc = None
+            return
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+        t = time.time()
+        while not self.lines and time.time() - t < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def begin(self):
+        import datetime
+        self.t_begin = datetime.datetime.now()
+
+    def end(self):
+        import datetime
+        self.t_end = datetime.datetime.now()
 
     def stop(self):
+        import datetime
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)   # let the sample after the region arrive
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=10)
+            self.proc.wait(timeout=10)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        rows = []
+        for line in list(self.lines):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-                power.append(float(f[3]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(f[2]), float(f[3]), float(f[4]), f[6:10]))
             except ValueError:
                 continue
-            for n, val in zip(names, f[5:9]):
+        pad = datetime.timedelta(milliseconds=100)
+        inside = [r for r in rows if self.t_begin and self.t_end and self.t_begin - pad <= r[0] <= self.t_end + pad]
+        used = inside
+        if not inside and rows and self.t_begin:
+            used = [min(rows, key=lambda r: abs((r[0] - self.t_begin).total_seconds()))]
+        reasons = set()
+        for r in used:
+            for n, val in zip(self.NAMES, r[4]):
                 if val.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
+        return {"sm_mhz": statistics.median(r[1] for r in used) if used else None,
+                "sm_max_mhz": max(r[2] for r in used) if used else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "samples_note": None if inside else "timed region shorter than the 50 ms sampling period: "
+                                                    "nearest sample reported",
+                "power_w_max": max(r[3] for r in used) if used else None}
 
 
 # ------------------------------------------------------------ roofline
@@ -264,11 +300,13 @@ def run_ours(args, rank, local, world, pg):
     launches0 = llsa.kernel_launches()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    clocks.begin()
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    clocks.end()
     launches = llsa.kernel_launches() - launches0
     barrier(pg)
     clk = clocks.stop()

@@ -495,12 +495,11 @@ cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, con
                                  const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                  const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                  void* dv, void* workspace, cudaStream_t s) {
-  size_t dsz = ((size_t)g.BH * g.N * sizeof(float) + 255) & ~(size_t)255;
-  size_t pyr = ((size_t)g.pyr_off[g.L + 1] * sizeof(float) + 255) & ~(size_t)255;
-  float* Dws = (float*)workspace;
-  float* dPK = (float*)((char*)workspace + dsz);
-  float* dPV = (float*)((char*)workspace + dsz + pyr);
-  cudaError_t e = cudaMemsetAsync(dPK, 0, 2 * pyr, s);
+  const BwdWorkspace ws = carve_bwd_workspace(g, workspace);
+  float* Dws = ws.D;
+  float* dPK = ws.dPK;
+  float* dPV = ws.dPV;
+  cudaError_t e = cudaMemsetAsync(dPK, 0, 2 * bwd_pyr_bytes(g), s);
   if (e != cudaSuccess) return e;
   if (g.bf16)
     return bwd_simt_any<__nv_bfloat16>(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, dq, dk, dv, Dws, dPK,

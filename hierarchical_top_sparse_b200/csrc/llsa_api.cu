@@ -98,6 +98,8 @@ cudaError_t launch_attn_bwd(const Geo& g, const void* q, const void* k, const vo
                             const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                             const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                             void* dv, void* workspace, cudaStream_t s) {
+  if (attn_bwd_mma_supported(g))
+    return launch_attn_bwd_mma(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, dq, dk, dv, workspace, s);
   return launch_attn_bwd_simt(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, dq, dk, dv, workspace, s);
 }
 

@@ -66,6 +66,11 @@ cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, con
                                  void* dv, void* workspace, cudaStream_t s);
 
 // Tensor-core attention kernels (bf16, d = 64, B = 16).
+bool attn_bwd_mma_supported(const Geo& g);
+cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, const void* v, const void* o,
+                                const void* dO, const float* lse, const float* pyrK, const float* pyrV,
+                                const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
+                                void* dv, void* workspace, cudaStream_t s);
 bool attn_fwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
@@ -78,13 +83,32 @@ cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows);
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
 
 // Workspace of the backward pass: D [BH][N] fp32, then the fp32 level gradients
-// of the pooled K and of the pooled V (each a pyramid).
+// of the pooled K and of the pooled V (each a pyramid), then a work counter.
+struct BwdWorkspace {
+  float* D;
+  float* dPK;
+  float* dPV;
+  int* counter;
+  size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counter)
+};
+
+inline size_t bwd_pyr_bytes(const Geo& g) {
+  return ((size_t)g.pyr_off[g.L + 1] * sizeof(float) + 255) & ~(size_t)255;
+}
+
 inline size_t bwd_workspace_bytes(const Geo& g) {
   size_t dsz = (size_t)g.BH * g.N * sizeof(float);
   dsz = (dsz + 255) & ~(size_t)255;
-  size_t pyr = (size_t)g.pyr_off[g.L + 1] * sizeof(float);
-  pyr = (pyr + 255) & ~(size_t)255;
-  return dsz + 2 * pyr;
+  return dsz + 2 * bwd_pyr_bytes(g) + 256;
+}
+
+inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
+  const size_t dsz = ((size_t)g.BH * g.N * sizeof(float) + 255) & ~(size_t)255;
+  const size_t pyr = bwd_pyr_bytes(g);
+  char* b = static_cast<char*>(workspace);
+  return BwdWorkspace{reinterpret_cast<float*>(b), reinterpret_cast<float*>(b + dsz),
+                      reinterpret_cast<float*>(b + dsz + pyr), reinterpret_cast<int*>(b + dsz + 2 * pyr),
+                      2 * pyr + sizeof(int)};
 }
 
 // ------------------------------------------------------------ device helpers
