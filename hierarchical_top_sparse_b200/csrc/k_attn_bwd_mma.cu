@@ -102,6 +102,11 @@ struct QSmem {
 
 using QRing = Ring<QR, QSLOT, QEXTRA>;
 
+// Column skew of row r of the pooled-gradient sums (element (r, c) sits at
+// column (c + skew(r & 7)) & 63): the 32 lanes of one atomic add of a C tile
+// (rows gq, columns 2 tq4 + const) then hit 32 different banks.
+__device__ __forceinline__ int acc_skew(int r7) { return 8 * ((r7 >> 1) & 3) + (r7 & 1); }
+
 // Row statistics of one query block for the lane's two C-tile rows (gq, gq + 8).
 struct RowStats {
   float lse2[2];   // LSE in the log2 domain
@@ -165,9 +170,10 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
   }
   __syncthreads();
 
-  const int g_begin = (int)(((int64_t)ngroups * blockIdx.x) / gridDim.x);
-  const int g_end = (int)(((int64_t)ngroups * (blockIdx.x + 1)) / gridDim.x);
-  const int nunits = 2 * (g_end - g_begin);
+  // Groups go to CTAs with a grid stride, so that the CTAs in flight work on
+  // neighbouring groups of one (batch, head) slice and share its K/V in L2.
+  const int ng_cta = ngroups > (int)blockIdx.x ? (ngroups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int nunits = 2 * ng_cta;
   QRing ring{s.ring[warp][0], s.full[warp], &s.meta[warp][0][0], 0u, 0u};
   if (lane == 0) {
     ptx::prefetch_tmap(&tq);
@@ -179,10 +185,10 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
 
   // ---------------------------------------------------------------- producer
   // The warp's elements, in order: for every unit u (query block
-  // (g_begin + u / 2) * 16 + 2 * warp + u % 2), a header (its Q, dO, O tiles
+  // (blockIdx.x + (u / 2) * gridDim.x) * 16 + 2 * warp + u % 2), a header (its Q, dO, O tiles
   // and LSE row) and then its K_1 picked K/V blocks.
   auto unit_block = [&](int u) -> int64_t {
-    return (int64_t)(g_begin + (u >> 1)) * GB + 2 * warp + (u & 1);
+    return ((int64_t)blockIdx.x + (int64_t)(u >> 1) * gridDim.x) * GB + 2 * warp + (u & 1);
   };
   auto pick_window = [&](int u, int j0) -> int {
     if (u >= nunits) return -1;
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
   };
 
   // ---------------------------------------------------------------- consumer
-  for (int gi = g_begin; gi < g_end; ++gi) {
+  for (int gi = blockIdx.x; gi < ngroups; gi += gridDim.x) {
     const int64_t a0g = (int64_t)gi * GB;
     const int64_t bh = a0g / g.n[1];
     const int a0 = (int)(a0g - bh * g.n[1]);
@@ -348,24 +354,38 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
         tiles::transpose_a(t, dsa);
         tiles::zero_acc(part);
         tiles::mma_ab(part, t, qtile, 0, lane);
+        const bool v0 = k0 + gq < nc, v1 = k0 + gq + 8 < nc;   // padding rows add nothing
+        const int sk = acc_skew(gq);
+        float* rk0 = s.accK + (k0 + gq) * 64;
+        float* rk1 = rk0 + 8 * 64;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int c = j * 8 + 2 * tq4;
-          atomicAdd(&s.accK[(k0 + gq) * 64 + c], part[j][0]);
-          atomicAdd(&s.accK[(k0 + gq) * 64 + c + 1], part[j][1]);
-          atomicAdd(&s.accK[(k0 + gq + 8) * 64 + c], part[j][2]);
-          atomicAdd(&s.accK[(k0 + gq + 8) * 64 + c + 1], part[j][3]);
+          const int c = j * 8 + 2 * tq4 + sk;
+          if (v0) {
+            atomicAdd(rk0 + (c & 63), part[j][0]);
+            atomicAdd(rk0 + ((c + 1) & 63), part[j][1]);
+          }
+          if (v1) {
+            atomicAdd(rk1 + (c & 63), part[j][2]);
+            atomicAdd(rk1 + ((c + 1) & 63), part[j][3]);
+          }
         }
         tiles::transpose_a(t, pa);
         tiles::zero_acc(part);
         tiles::mma_ab(part, t, dotile, 0, lane);
+        float* rv0 = s.accV + (k0 + gq) * 64;
+        float* rv1 = rv0 + 8 * 64;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int c = j * 8 + 2 * tq4;
-          atomicAdd(&s.accV[(k0 + gq) * 64 + c], part[j][0]);
-          atomicAdd(&s.accV[(k0 + gq) * 64 + c + 1], part[j][1]);
-          atomicAdd(&s.accV[(k0 + gq + 8) * 64 + c], part[j][2]);
-          atomicAdd(&s.accV[(k0 + gq + 8) * 64 + c + 1], part[j][3]);
+          const int c = j * 8 + 2 * tq4 + sk;
+          if (v0) {
+            atomicAdd(rv0 + (c & 63), part[j][0]);
+            atomicAdd(rv0 + ((c + 1) & 63), part[j][1]);
+          }
+          if (v1) {
+            atomicAdd(rv1 + (c & 63), part[j][2]);
+            atomicAdd(rv1 + ((c + 1) & 63), part[j][3]);
+          }
         }
       }
       __syncwarp();
@@ -425,8 +445,9 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
         if (tok < 0) continue;
         const int l = s.crow_l[row];
         const int64_t off = g.pyr_off[l] + (bh * g.n[l] + tok) * 64 + c;
-        atomicAdd(dPK + off, s.accK[e] * g.scale);
-        atomicAdd(dPV + off, s.accV[e]);
+        const int sidx = row * 64 + ((c + acc_skew(row & 7)) & 63);
+        atomicAdd(dPK + off, s.accK[sidx] * g.scale);
+        atomicAdd(dPV + off, s.accV[sidx]);
       }
     }
   }

@@ -281,9 +281,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
   }
   __syncthreads();
 
-  // every CTA takes a contiguous range of groups (spatial neighbours)
-  const int g_begin = (int)(((int64_t)ngroups * blockIdx.x) / gridDim.x);
-  const int g_end = (int)(((int64_t)ngroups * (blockIdx.x + 1)) / gridDim.x);
+  // Pairs of groups (the 16 blocks under one level-2 token) go to CTAs with a
+  // grid stride: the CTAs in flight work on neighbouring groups of one
+  // (batch, head) slice and share its K/V in L2.  Iteration `it` of this CTA
+  // takes group group_of(it); the sequence is increasing.
+  auto group_of = [&](int it) -> int {
+    return 2 * ((int)blockIdx.x + (it >> 1) * (int)gridDim.x) + (it & 1);
+  };
 
   if (warp == TMA_WARP) {
     // ----------------------------------------- union of the picks, TMA loads
@@ -300,14 +304,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
       return idx + g.idx_off[1] + ((int64_t)bh * g.n[1] + a0) * K1;   // the G lists are consecutive
     };
     int nx0 = 0x7fffffff, nx1 = 0x7fffffff;   // next group's picks (small case), prefetched
-    if (small && g_begin < g_end) {
-      const int32_t* pk = pick_ptr(g_begin);
+    if (small && group_of(0) < ngroups) {
+      const int32_t* pk = pick_ptr(group_of(0));
       if (2 * lane < np) nx0 = pk[2 * lane];
       if (2 * lane + 1 < np) nx1 = pk[2 * lane + 1];
     }
     uint32_t ring_pos = 0;
     int it = 0;
-    for (int gi = g_begin; gi < g_end; ++gi, ++it) {
+    for (int gi = group_of(0); gi < ngroups; gi = group_of(++it)) {
       const int b = it % NBUF;
       const uint32_t use = (uint32_t)(it / NBUF);
       const int bh = gi / groups_per_slice;
@@ -327,8 +331,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
         o0 = x0;
         o1 = x1;
         nx0 = nx1 = 0x7fffffff;
-        if (gi + 1 < g_end) {                 // prefetch the next group's picks
-          const int32_t* pk = pick_ptr(gi + 1);
+        if (group_of(it + 1) < ngroups) {     // prefetch the next group's picks
+          const int32_t* pk = pick_ptr(group_of(it + 1));
           if (2 * lane < np) nx0 = pk[2 * lane];
           if (2 * lane + 1 < np) nx1 = pk[2 * lane + 1];
         }
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
       for (uint32_t p = lo2 + lane; p < ring_pos; p += 32)
         ptx::mbar_wait_bounded(&s.full[p % SLOTS], (p / SLOTS) & 1, kWaitLimitNs);
       if (lane == 0)
-        for (int j = it > NBUF - 1 ? it - NBUF + 1 : 0; j <= it && j < g_end - g_begin; ++j)
+        for (int j = it > NBUF - 1 ? it - NBUF + 1 : 0; j <= it && group_of(j) < ngroups; ++j)
           ptx::mbar_wait_bounded(&s.qfull[j % NBUF], (j / NBUF) & 1, kWaitLimitNs);
     }
     return;
@@ -451,7 +455,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
   uint32_t cphase = 0;
   int64_t last_parent = -1;
   int it = 0;
-  for (int gi = g_begin; gi < g_end; ++gi, ++it) {
+  for (int gi = group_of(0); gi < ngroups; gi = group_of(++it)) {
     const int b = it % NBUF;
     const uint32_t use = (uint32_t)(it / NBUF);
     const int bh = gi / groups_per_slice;
@@ -665,7 +669,8 @@ cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int gps = g.n[1] / fwdmma::G;
   const int ngroups = g.BH * gps;
-  const int grid = ngroups < sms ? ngroups : sms;
+  const int npairs = (ngroups + 1) / 2;
+  const int grid = npairs < sms ? npairs : sms;
   fwdmma::attn_fwd_mma_kernel<<<grid, fwdmma::THREADS, smem, s>>>(g, tq, tk, tv, pyrK, pyrV, idx,
                                                                   (__nv_bfloat16*)o, lse, device_error_word(), gps,
                                                                   ngroups);

@@ -76,10 +76,12 @@ __device__ __forceinline__ void load4(const __nv_bfloat16* p, float* v) {
 // Level l from level l-1: P_l[j] = (1/B) sum_{r<B} P_{l-1}[j*B + r]
 // (hierarchical compression, Trainable Log-linear Sparse Attention summary §三).
 // One thread per (slice, pooled token, 4 channels); fp32 accumulation in the
-// order r = 0..B-1.
-template <typename Tin>
-__global__ void pool_level_kernel(const Tin* __restrict__ in, float* __restrict__ out, int64_t n_out, int d,
-                                  int B, int64_t total) {
+// order r = 0..B-1.  With B a compile-time constant all B row loads of a
+// thread are in flight at once.
+template <typename Tin, int BC>
+__global__ void pool_level_kernel(const Tin* __restrict__ in, float* __restrict__ out, int d, int Brt,
+                                  int64_t total) {
+  const int B = BC > 0 ? BC : Brt;
   int c4n = d / 4;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
@@ -87,29 +89,48 @@ __global__ void pool_level_kernel(const Tin* __restrict__ in, float* __restrict_
     int c = (int)(e - tok * c4n) * 4;
     const Tin* src = in + tok * B * d + c;       // rows j*B .. j*B+B-1 of the same slice
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < B; ++r) {
-      float v[4];
-      load4(src + (int64_t)r * d, v);
-      acc[0] += v[0]; acc[1] += v[1]; acc[2] += v[2]; acc[3] += v[3];
+    if (BC > 0) {
+      float v[BC > 0 ? BC : 1][4];
+#pragma unroll
+      for (int r = 0; r < BC; ++r) load4(src + (int64_t)r * d, v[r]);
+#pragma unroll
+      for (int r = 0; r < BC; ++r) {
+        acc[0] += v[r][0]; acc[1] += v[r][1]; acc[2] += v[r][2]; acc[3] += v[r][3];
+      }
+    } else {
+      for (int r = 0; r < B; ++r) {
+        float v[4];
+        load4(src + (int64_t)r * d, v);
+        acc[0] += v[0]; acc[1] += v[1]; acc[2] += v[2]; acc[3] += v[3];
+      }
     }
     float4 o = make_float4(acc[0] / B, acc[1] / B, acc[2] / B, acc[3] / B);
     *reinterpret_cast<float4*>(out + tok * d + c) = o;
   }
-  (void)n_out;
+}
+
+template <typename Tin>
+static void pool_launch(const Tin* in, float* out, const Geo& g, int64_t total, cudaStream_t s) {
+  const int grid = grid_for(total, 256);
+  if (g.B == 16)
+    pool_level_kernel<Tin, 16><<<grid, 256, 0, s>>>(in, out, g.d, g.B, total);
+  else if (g.B == 4)
+    pool_level_kernel<Tin, 4><<<grid, 256, 0, s>>>(in, out, g.d, g.B, total);
+  else
+    pool_level_kernel<Tin, 0><<<grid, 256, 0, s>>>(in, out, g.d, g.B, total);
 }
 
 cudaError_t launch_pool(const Geo& g, const void* x, float* pyr, cudaStream_t s) {
   for (int l = 1; l <= g.L; ++l) {
     int64_t total = (int64_t)g.BH * g.n[l] * (g.d / 4);
     float* out = pyr + g.pyr_off[l];
-    int grid = grid_for(total, 256);
     if (l == 1) {
       if (g.bf16)
-        pool_level_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)x, out, g.n[l], g.d, g.B, total);
+        pool_launch((const __nv_bfloat16*)x, out, g, total, s);
       else
-        pool_level_kernel<float><<<grid, 256, 0, s>>>((const float*)x, out, g.n[l], g.d, g.B, total);
+        pool_launch((const float*)x, out, g, total, s);
     } else {
-      pool_level_kernel<float><<<grid, 256, 0, s>>>(pyr + g.pyr_off[l - 1], out, g.n[l], g.d, g.B, total);
+      pool_launch((const float*)(pyr + g.pyr_off[l - 1]), out, g, total, s);
     }
     note_launches(1);
     cudaError_t e = cudaGetLastError();

@@ -99,8 +99,147 @@ __global__ void select_level_kernel(Geo g, int l, const float* __restrict__ pyrQ
   }
 }
 
+// ------------------------------------------------ child search, one CTA per parent
+//
+// The B sibling query tokens under one level-(l+1) token share their
+// candidates (the B children of each of the parent's picks), so one CTA
+// loads those candidate rows once into shared memory and scores the whole
+// B x (K_{l+1} B) tile: every thread a 4 x 4 register tile of scores, each a
+// sequential fp32 FMA chain over d (the same rounding as the one-warp kernel
+// above).  Then one warp per query token takes K_l rounds of a warp-wide max
+// over 64-bit keys held in registers and writes the picks in ascending order.
+namespace selchild {
+constexpr int THREADS = 128;
+constexpr int NC = 128;        // candidates per parent, at most
+constexpr int QB = 16;         // sibling query tokens (B)
+constexpr int LD = 68;         // padded row length (floats): conflict-free 16-byte reads
+}
+
+__global__ void __launch_bounds__(selchild::THREADS) select_children_kernel(Geo g, int l,
+                                                                            const float* __restrict__ pyrQ,
+                                                                            const float* __restrict__ pyrK,
+                                                                            int32_t* __restrict__ idx) {
+  using namespace selchild;
+  __shared__ __align__(16) float ks[NC * LD];
+  __shared__ __align__(16) float qs[QB * LD];
+  __shared__ float sc[QB][NC];
+  __shared__ int cid[NC];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nl = g.n[l], np = g.n[l + 1];
+  const int bh = blockIdx.x / np;
+  const int par = blockIdx.x - bh * np;
+  const int Kp = g.Kl[l + 1], Kl = g.Kl[l];
+  const int ncand = Kp * QB;
+  const int32_t* plist = idx + g.idx_off[l + 1] + ((int64_t)bh * np + par) * Kp;
+  const float* kbase = pyrK + g.pyr_off[l] + (int64_t)bh * nl * 64;
+  const float* qbase = pyrQ + g.pyr_off[l] + ((int64_t)bh * nl + (int64_t)par * QB) * 64;
+
+  // candidate ids (position m = pick m / B, child m % B), then the rows
+  if (tid < NC) {
+    int c = -1;
+    if (tid < ncand) {
+      const int pc = plist[tid / QB];
+      c = (pc >= 0 && pc < np) ? pc * QB + tid % QB : -1 - (pc * QB + tid % QB);   // < 0: parent corrupted
+    }
+    cid[tid] = c;
+  }
+  for (int e = tid; e < QB * 16; e += THREADS) {
+    const int r = e >> 4, c4 = (e & 15) * 4;
+    *reinterpret_cast<float4*>(&qs[r * LD + c4]) = *reinterpret_cast<const float4*>(qbase + r * 64 + c4);
+  }
+  __syncthreads();
+  for (int e = tid; e < NC * 16; e += THREADS) {
+    const int m = e >> 4, c4 = (e & 15) * 4;
+    const int c = cid[m];
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c >= 0) v = *reinterpret_cast<const float4*>(kbase + (int64_t)c * 64 + c4);
+    *reinterpret_cast<float4*>(&ks[m * LD + c4]) = v;
+  }
+  __syncthreads();
+
+  // scores: warp w takes query rows 4w..4w+3, lane the candidates lane + 32 j
+  {
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int e = 0; e < 64; e += 4) {
+      float4 qv[4], kv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(&qs[(warp * 4 + i) * LD + e]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) kv[j] = *reinterpret_cast<const float4*>(&ks[(lane + 32 * j) * LD + e]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sc[warp * 4 + i][lane + 32 * j] = acc[i][j];
+  }
+  __syncwarp();
+
+  // top-K_l per query row; rows 4w..4w+3 were scored by this warp
+  for (int i = 0; i < 4; ++i) {
+    const int r = warp * 4 + i;
+    uint64_t key[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = lane + 32 * j;
+      if (m >= ncand)
+        key[j] = 0;
+      else if (cid[m] < 0)
+        key[j] = 1ull << 32;          // parent corrupted: the candidate never wins
+      else
+        key[j] = ((uint64_t)orderable(sc[r][m]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)m);
+    }
+    unsigned taken = 0;
+    for (int k = 0; k < Kl; ++k) {
+      uint64_t best = key[0];
+#pragma unroll
+      for (int j = 1; j < 4; ++j) best = key[j] > best ? key[j] : best;
+      best = warp_max_u64(best);
+      const int m = (int)(0xffffffffu - (uint32_t)best);
+      if ((m & 31) == lane) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j == (m >> 5)) key[j] = 0;
+        taken |= 1u << (m >> 5);
+      }
+    }
+    int32_t* out = idx + g.idx_off[l] + ((int64_t)bh * nl + (int64_t)par * QB + r) * Kl;
+    int written = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool t = (taken >> j) & 1u;
+      const unsigned bal = __ballot_sync(0xffffffffu, t);
+      if (t) {
+        const int m = lane + 32 * j;
+        const int c = cid[m];
+        out[written + __popc(bal & ((1u << lane) - 1u))] = c >= 0 ? c : -1 - c;
+      }
+      written += __popc(bal);
+    }
+  }
+}
+
 cudaError_t launch_select_level(const Geo& g, int level, const float* pyrQ, const float* pyrK, int32_t* idx,
                                 cudaStream_t s) {
+  if (level < g.L && g.d == 64 && g.B == selchild::QB && g.Kl[level + 1] * g.B <= selchild::NC &&
+      g.Kl[level] < g.Kl[level + 1] * g.B) {
+    const int64_t parents = (int64_t)g.BH * g.n[level + 1];
+    select_children_kernel<<<(unsigned)parents, selchild::THREADS, 0, s>>>(g, level, pyrQ, pyrK, idx);
+    note_launches(1);
+    return cudaGetLastError();
+  }
   const int nl = g.n[level];
   const int ncand = level == g.L ? nl : g.Kl[level + 1] * g.B;
   int warps = 8;
