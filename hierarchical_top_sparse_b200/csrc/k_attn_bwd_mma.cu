@@ -9,10 +9,9 @@
 //    one level-2 token, so a CTA takes one level-2 token at a time, reduces
 //    their gradients (scale * dS^T Q and P^T dO) in shared memory and adds
 //    them with one fp32 atomic per (pooled token, channel).
-//  * key-major pass, per fine key block (16 keys), over the query blocks of
-//    its level-1 CSC list: dV += P^T dO, dK += scale * dS^T Q; then the
-//    pooled-key gradients of levels >= 2 are spread back over the B^l tokens
-//    each pooled token averages (divided by B^l).
+//  * key-major pass (k_attn_bwd_kv_tc.cu, on tcgen05), per fine key block,
+//    over the query blocks of its level-1 CSC list: dV, dK, and the pooled-key
+//    gradients of levels >= 2 spread back over the B^l tokens they average.
 //
 // A level-1 pooled token is the mean of the 16 keys of the block it stands
 // for, and the queries that attend it are exactly those that picked that
@@ -23,13 +22,11 @@
 //
 // Every warp streams its own tiles through a small ring of shared-memory
 // slots filled by TMA (2-D tile loads of 2 KB blocks with the 128-byte
-// swizzle; 1-D bulk loads of 64-byte LSE / D rows), a few elements ahead of
-// the one it computes, so list lengths are unbounded.  Work: query-major,
-// static (16 query blocks per CTA step, 2 per warp); key-major, chunks of
-// CHUNK key blocks taken from a global counter, because the CSC lists have
-// very uneven lengths.  Every wait is bounded; a warp that gives up sets the
-// device error word, stops computing and, before it exits, waits (bounded)
-// for the copies it issued.
+// swizzle; a 1-D bulk load of the 64-byte LSE row), a few elements ahead of
+// the one it computes, so list lengths are unbounded.  Query blocks are
+// assigned statically (16 per CTA step, 2 per warp).  Every wait is bounded;
+// a warp that gives up sets the device error word, stops computing and,
+// before it exits, waits (bounded) for the copies it issued.
 #include <math.h>
 
 #include "llsa_internal.cuh"
@@ -43,8 +40,6 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: a wait this long mean
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int GB = 16;        // query blocks per query-major CTA step (one level-2 token)
 constexpr int COARSE = 32;    // pooled keys of levels >= 2 per query block, at most
-
-enum : int { kEnd = 0, kHeader = 1, kEntry = 2 };
 
 // ------------------------------------------------------ per-warp TMA ring
 
@@ -454,262 +449,6 @@ __global__ void __launch_bounds__(QW * 32, 1) attn_bwd_q_mma_kernel(
   if (!live) ring.drain();
 }
 
-// ------------------------------------------------------ key-major pass
-
-constexpr int KW = 12;         // warps per CTA
-constexpr int KR = 3;          // ring slots per warp
-constexpr int KSLOT = 5120;    // header: K, V tiles; entry: Q, dO tiles + LSE and D rows
-constexpr int KEXTRA = 4096;
-constexpr int CHUNK = 4;       // key blocks taken from the work counter at a time
-
-struct KSmem {
-  alignas(1024) unsigned char ring[KW][KR][KSLOT];
-  int meta[KW][KR][4];
-  alignas(8) uint64_t full[KW][KR];
-};
-
-using KRing = Ring<KR, KSLOT, KEXTRA>;
-
-__global__ void __launch_bounds__(KW * 32, 1) attn_bwd_kv_mma_kernel(
-    const __grid_constant__ Geo g, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-    const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo, const float* __restrict__ lse,
-    const float* __restrict__ Dws, const int32_t* __restrict__ offs, const int32_t* __restrict__ qlist,
-    const float* __restrict__ dPK, const float* __restrict__ dPV, __nv_bfloat16* __restrict__ dk,
-    __nv_bfloat16* __restrict__ dv, int* counter, int* err) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  KSmem& s = *reinterpret_cast<KSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq4 = lane & 3;
-  const int n1 = g.n[1];
-  const int64_t slice_entries = (int64_t)n1 * g.Kl[1];   // level-1 CSC entries per slice
-  const int64_t total = (int64_t)g.BH * n1;               // fine key blocks
-  const float log2B = log2f((float)g.B);
-  const float sc2 = g.scale * kLog2e;
-  const bool enrich1 = g.emask & 1u;
-
-  if (lane == 0)
-    for (int i = 0; i < KR; ++i) ptx::mbar_init(&s.full[warp][i], 1);
-  if (lane == 0) {
-    ptx::fence_mbar_init();
-    ptx::prefetch_tmap(&tk);
-    ptx::prefetch_tmap(&tv);
-    ptx::prefetch_tmap(&tq);
-    ptx::prefetch_tmap(&tdo);
-  }
-  __syncwarp();
-  KRing ring{s.ring[warp][0], s.full[warp], &s.meta[warp][0][0], 0u, 0u};
-
-  // ---------------------------------------------------------------- producer
-  // Elements: for every key block taken (CHUNK at a time from the counter), a
-  // header (its K and V tiles) and then one element per entry of its CSC
-  // list (the query block's Q and dO tiles, LSE and D rows); kEnd when the
-  // counter runs past the last block.
-  int64_t cb = 0, ce = 0;        // current chunk [cb, ce)
-  int64_t ukb = 0;               // producer's current key block
-  int pj = -1, ust = 0, ulen = 0;
-  int ow = 0;                    // lane l <= CHUNK: list start of key block cb + l (slice-local)
-  int wpos = -1, lw = -1;        // list window: lane l holds entry wpos + l of the chunk's slice
-  int nxt_l0 = 0;                // lane 0: start of the next chunk (counter value)
-  bool done = false, live = true;
-  if (lane == 0) nxt_l0 = atomicAdd(counter, CHUNK);
-
-  auto pump = [&]() {
-    while (live && !done && ring.can_issue()) {
-      const uint32_t i = ring.issued;
-      unsigned char* sl = ring.slot(i);
-      uint64_t* bar = ring.bar(i);
-      int* meta = ring.meta_of(i);
-      if (pj < 0 && ukb >= ce) {
-        // take the next chunk; ask for the one after it right away
-        cb = (int64_t)__shfl_sync(0xffffffffu, nxt_l0, 0);
-        if (cb >= total) {
-          if (lane == 0) {
-            meta[0] = kEnd;
-            ptx::mbar_arrive(bar);
-          }
-          __syncwarp();
-          ++ring.issued;
-          done = true;
-          break;
-        }
-        if (lane == 0) nxt_l0 = atomicAdd(counter, CHUNK);
-        ce = cb + CHUNK < total ? cb + CHUNK : total;
-        const int64_t bh = cb / n1;
-        const int kb0 = (int)(cb - bh * n1);
-        ow = lane <= (int)(ce - cb) ? offs[g.offs_off[1] + bh * (n1 + 1) + kb0 + lane] : 0;
-        ukb = cb;
-        wpos = -1;
-      }
-      const int64_t bh = ukb / n1;
-      if (pj < 0) {
-        ust = __shfl_sync(0xffffffffu, ow, (int)(ukb - cb));
-        ulen = __shfl_sync(0xffffffffu, ow, (int)(ukb - cb) + 1) - ust;
-        if (ulen < 0 || ust < 0 || ust + (int64_t)ulen > slice_entries) ulen = 0;   // never produced by the transpose
-        if (lane == 0) {
-          meta[0] = kHeader;
-          meta[1] = (int)ukb;
-          meta[2] = ulen;
-          ptx::fence_proxy_async();
-          const int row = (int)(ukb * 16);
-          ptx::mbar_arrive_expect_tx(bar, 4096);
-          ptx::tma_load_2d(sl, &tk, 0, row, bar);
-          ptx::tma_load_2d(sl + 2048, &tv, 0, row, bar);
-        }
-        if (ulen == 0)
-          ++ukb;
-        else
-          pj = 0;
-      } else {
-        const int pos = ust + pj;
-        if (wpos < 0 || pos < wpos || pos >= wpos + 32) {
-          wpos = pos;
-          lw = (int64_t)wpos + lane < slice_entries ? qlist[g.idx_off[1] + bh * slice_entries + wpos + lane] : -1;
-        }
-        const int a = __shfl_sync(0xffffffffu, lw, pos - wpos);
-        const bool ok = a >= 0 && a < n1;
-        if (lane == 0) {
-          meta[0] = kEntry;
-          meta[1] = ok ? 1 : 0;
-          ptx::fence_proxy_async();
-          if (ok) {
-            const int64_t row = (bh * n1 + a) * 16;
-            ptx::mbar_arrive_expect_tx(bar, 4096 + 128);
-            ptx::tma_load_2d(sl, &tq, 0, (int)row, bar);
-            ptx::tma_load_2d(sl + 2048, &tdo, 0, (int)row, bar);
-            ptx::bulk_load(sl + KEXTRA, lse + row, 64, bar);
-            ptx::bulk_load(sl + KEXTRA + 64, Dws + row, 64, bar);
-          } else {
-            ptx::mbar_arrive(bar);   // a query id outside its level: nothing to load
-          }
-        }
-        if (++pj == ulen) {
-          pj = -1;
-          ++ukb;
-        }
-      }
-      __syncwarp();
-      ++ring.issued;
-    }
-  };
-
-  // ---------------------------------------------------------------- consumer
-  uint32_t kfr[4][4], vfr[4][4];
-  float dka[8][4], dva[8][4];
-  int64_t ckb = -1;
-  int remaining = 0;
-  while (true) {
-    pump();
-    if (!live) break;
-    if (!ring.wait_next()) {
-      live = false;
-      report(err, 22);
-      break;
-    }
-    const uint32_t i = ring.consumed;
-    const int* meta = ring.meta_of(i);
-    const int kind = meta[0];
-    if (kind == kEnd) {
-      __syncwarp();
-      ++ring.consumed;
-      break;
-    }
-    if (kind == kHeader) {
-      ckb = meta[1];
-      remaining = meta[2];
-      tiles::load_a(kfr, ring.tile(i, 0), lane);
-      tiles::load_a(vfr, ring.tile(i, 1), lane);
-      tiles::zero_acc(dka);
-      tiles::zero_acc(dva);
-    } else {
-      if (meta[1]) {
-        const uint32_t qtile = ring.tile(i, 0), dotile = ring.tile(i, 1);
-        const float* ex = ring.extra(i);
-        // S^T and dP^T: rows = the block's keys, columns = the entry's queries
-        float st[2][4], dpt[2][4];
-        tiles::mma_abt(st, kfr, qtile, 0, lane);
-        tiles::mma_abt(dpt, vfr, dotile, 0, lane);
-        float l2[2][2], Dq[2][2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            const int qc = j * 8 + 2 * tq4 + b;
-            l2[j][b] = ex[qc] * kLog2e;
-            Dq[j][b] = ex[16 + qc];
-          }
-        float p[2][4], ds[2][4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            p[j][e] = exp2f(st[j][e] * sc2 - l2[j][e & 1]);
-            ds[j][e] = p[j][e] * (dpt[j][e] - Dq[j][e & 1]);
-          }
-        if (enrich1) {
-          // per query (column): the block's pooled level-1 token
-#pragma unroll
-          for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-              const float zs = tiles::column_sum8(st[j][b] + st[j][b + 2]);
-              const float dps = tiles::column_sum8(dpt[j][b] + dpt[j][b + 2]);
-              const float pc = exp2f(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2[j][b]);
-              const float dsc = pc * (dps * (1.f / 16.f) - Dq[j][b]);
-              p[j][b] += pc * (1.f / 16.f);
-              p[j][b + 2] += pc * (1.f / 16.f);
-              ds[j][b] += dsc * (1.f / 16.f);
-              ds[j][b + 2] += dsc * (1.f / 16.f);
-            }
-        }
-        uint32_t pa[4], dsa[4];
-        tiles::pack_a(pa, p);
-        tiles::pack_a(dsa, ds);
-        tiles::mma_ab(dva, pa, dotile, 0, lane);
-        tiles::mma_ab(dka, dsa, qtile, 0, lane);
-      }
-      --remaining;
-    }
-    __syncwarp();
-    ++ring.consumed;
-    if (remaining > 0) continue;
-
-    // ------------------------------------------- epilogue of key block ckb
-    const int64_t bh = ckb / n1;
-    const int64_t t0 = (ckb - bh * n1) * 16;   // first fine token of the block
-    float ak[8][2], av[8][2];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) ak[j][0] = ak[j][1] = av[j][0] = av[j][1] = 0.f;
-    for (int l = 2; l <= g.L; ++l) {
-      if (!((g.emask >> (l - 1)) & 1u)) continue;
-      const int64_t off = g.pyr_off[l] + (bh * g.n[l] + t0 / g.Bl[l]) * 64;
-      const float inv = 1.f / (float)g.Bl[l];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = j * 8 + 2 * tq4;
-        const float2 kk = *reinterpret_cast<const float2*>(dPK + off + c);
-        const float2 vv = *reinterpret_cast<const float2*>(dPV + off + c);
-        ak[j][0] = fmaf(kk.x, inv, ak[j][0]);
-        ak[j][1] = fmaf(kk.y, inv, ak[j][1]);
-        av[j][0] = fmaf(vv.x, inv, av[j][0]);
-        av[j][1] = fmaf(vv.y, inv, av[j][1]);
-      }
-    }
-    const int64_t r0 = ckb * 16 + gq;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = j * 8 + 2 * tq4;
-      *reinterpret_cast<uint32_t*>(dk + r0 * 64 + c) =
-          ptx::pack_bf16(fmaf(dka[j][0], g.scale, ak[j][0]), fmaf(dka[j][1], g.scale, ak[j][1]));
-      *reinterpret_cast<uint32_t*>(dk + (r0 + 8) * 64 + c) =
-          ptx::pack_bf16(fmaf(dka[j][2], g.scale, ak[j][0]), fmaf(dka[j][3], g.scale, ak[j][1]));
-      *reinterpret_cast<uint32_t*>(dv + r0 * 64 + c) = ptx::pack_bf16(dva[j][0] + av[j][0], dva[j][1] + av[j][1]);
-      *reinterpret_cast<uint32_t*>(dv + (r0 + 8) * 64 + c) =
-          ptx::pack_bf16(dva[j][2] + av[j][0], dva[j][3] + av[j][1]);
-    }
-  }
-  if (!live) ring.drain();
-}
-
 }  // namespace bwdmma
 
 // ------------------------------------------------------------------ launch
@@ -759,11 +498,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwdmma::attn_bwd_kv_mma_kernel<<<sms, bwdmma::KW * 32, ksmem, s>>>(
-      g, tk, tv, tq, tdo, lse, ws.D, offs, qlist, ws.dPK, ws.dPV, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, ws.counter,
-      err);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_attn_bwd_kv_tc(g, tk, tv, tq, tdo, lse, ws.D, offs, qlist, ws.dPK, ws.dPV, dk, dv, ws.counter, s);
 }
 
 }  // namespace llsa

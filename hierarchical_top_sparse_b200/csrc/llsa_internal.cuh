@@ -71,6 +71,10 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                 void* dv, void* workspace, cudaStream_t s);
+cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                                  const CUtensorMap& tdo, const float* lse, const float* D, const int32_t* offs,
+                                  const int32_t* qlist, const float* dPK, const float* dPV, void* dk, void* dv,
+                                  int* counter, cudaStream_t s);
 bool attn_fwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
