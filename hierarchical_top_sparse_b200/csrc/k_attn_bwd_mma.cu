@@ -481,11 +481,8 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   BwdWorkspace ws = carve_bwd_workspace(g, workspace);
   e = cudaMemsetAsync(ws.dPK, 0, ws.zero_bytes, s);   // pooled-key sums and the work counter
   if (e != cudaSuccess) return e;
-  const size_t qsmem = sizeof(bwdmma::QSmem) + 1024, ksmem = sizeof(bwdmma::KSmem) + 1024;
+  const size_t qsmem = sizeof(bwdmma::QSmem) + 1024;
   e = cudaFuncSetAttribute(bwdmma::attn_bwd_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(bwdmma::attn_bwd_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)ksmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -498,7 +495,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attn_bwd_kv_tc(g, tk, tv, tq, tdo, lse, ws.D, offs, qlist, ws.dPK, ws.dPV, dk, dv, ws.counter, s);
+  return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, ws.D, offs, qlist, ws.dPK, ws.dPV, dk, dv, ws.counter, s);
 }
 
 }  // namespace llsa

@@ -71,7 +71,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                 void* dv, void* workspace, cudaStream_t s);
-cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
                                   const CUtensorMap& tdo, const float* lse, const float* D, const int32_t* offs,
                                   const int32_t* qlist, const float* dPK, const float* dPV, void* dk, void* dv,
                                   int* counter, cudaStream_t s);
@@ -82,6 +82,8 @@ cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, cons
 // TMA descriptor of a [rows][64] bf16 token tensor, boxes of 16 rows x 64
 // columns (one 2 KB key or query block), 128-byte swizzle.
 cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows);
+// Same with boxes of `box_rows` rows (1..256).
+cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 // Largest candidate count the selection kernel keeps in shared memory.
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp

@@ -21,12 +21,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows) {
+  return make_token_map_box(map, base, rows, 16);
+}
+
+cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  if (((uintptr_t)base & 15u) != 0) return cudaErrorInvalidValue;
+  if (((uintptr_t)base & 15u) != 0 || box_rows < 1 || box_rows > 256) return cudaErrorInvalidValue;
   cuuint64_t dims[2] = {64, (cuuint64_t)rows};
   cuuint64_t strides[1] = {64 * sizeof(__nv_bfloat16)};
-  cuuint32_t box[2] = {64, 16};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
