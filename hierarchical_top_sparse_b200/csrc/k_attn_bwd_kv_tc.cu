@@ -27,10 +27,11 @@
 // pairs, computed and discarded.
 //
 // Warp roles, one CTA per SM:
-//   * warp 12, producer: takes key groups from a global counter, merges the
-//     group's 8 sorted CSC lists into the union, and loads every chunk (one
-//     lane per 2 KB tile) into one of NSLOT slots and every group's K and V
-//     (one 16 KB box each) into one of two key slots, all with TMA;
+//   * warp 12, producer: takes the CTA's key groups (grid stride, so that the
+//     CTAs in flight share neighbouring Q/dO tiles in L2), reads each group's
+//     union (prefetched two groups ahead), and loads every chunk (one lane
+//     per 2 KB tile) into one of NSLOT slots and every group's K and V (one
+//     16 KB box each) into one of two key slots, all with TMA;
 //   * warp 13, MMA: a converged warp whose elected lane issues the MMAs and
 //     commits them to mbarriers;
 //   * warps 0-7, softmax: warps w and w + 4 share TMEM lanes 32 (w % 4).. and
@@ -38,6 +39,12 @@
 //   * warps 8-11, epilogue.
 // Every hand-off is an mbarrier, every wait is bounded; on a timeout the
 // kernel sets the device error word and stops.
+//
+// The unions come from a pre-pass, kv_union_kernel: one warp per key group
+// merges the group's 8 sorted level-1 CSC lists and writes the union in
+// ascending query-block order, each entry (query block << 8) | pick mask,
+// into the group's own range of the CSC layout (a union is never longer than
+// the lists it merges).
 #include <math.h>
 #include <stddef.h>
 
@@ -55,8 +62,8 @@ constexpr int KG = 8;               // key blocks per group (128 keys)
 constexpr int NSLOT = 3;            // chunk slots
 constexpr int SOFT_WARPS = 8, PRODUCER_WARP = 12, MMA_WARP = 13;   // warps 8-11: epilogue
 constexpr int THREADS = 14 * 32;
-constexpr int TAKE = 2;             // key groups taken from the counter at a time
-constexpr int LISTCAP = 256;        // CSC entries of one take staged in shared memory
+constexpr int UNION_WARPS = 8;      // pre-pass: warps per block (one key group each)
+constexpr int UNION_CAP = 512;      // pre-pass: CSC entries of a group staged in shared memory
 constexpr int UPL = 4;              // pooled levels (2..5) whose gradients the epilogue keeps in registers
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 384;
@@ -90,8 +97,6 @@ struct Smem {
   alignas(1024) unsigned char pbuf[2 * 16384];
   alignas(1024) unsigned char sbuf[2 * 16384];
   Meta meta[NSLOT];
-  int list[LISTCAP];                           // producer: the CSC entries of the groups taken
-  int pend_q[CQ], pend_m[CQ];                  // producer: union members of the chunk being built
   alignas(8) uint64_t full[NSLOT], empty[NSLOT];
   uint64_t kfull[2], kempty[2];                // key slots: producer -> MMA, MMA -> producer
   uint64_t s_full, s_empty;                    // S / dP in TMEM: MMA -> softmax, softmax (8 warps) -> MMA
@@ -109,12 +114,73 @@ __device__ __forceinline__ void report(int* err, int code) {
   if (err) atomicExch(err, code);
 }
 
+// One warp per key group: the union of the 8 blocks' level-1 CSC lists (each
+// sorted ascending), in ascending order, each entry (query block << 8) | mask
+// where bit j says that the query block picked key block 8 g + j.  Written at
+// the group's own CSC range [offs(8 g), offs(8 g) + size); size in ucount[g].
+__global__ void __launch_bounds__(UNION_WARPS * 32) kv_union_kernel(Geo g, const int32_t* __restrict__ offs,
+                                                                    const int32_t* __restrict__ qlist,
+                                                                    int32_t* __restrict__ ulist,
+                                                                    int32_t* __restrict__ ucount, int ngroups) {
+  __shared__ int stage[UNION_WARPS][UNION_CAP];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gi = blockIdx.x * UNION_WARPS + warp;
+  if (gi >= ngroups) return;
+  const int n1 = g.n[1];
+  const int64_t slice_entries = (int64_t)n1 * g.Kl[1];
+  const int bh = gi * KG / n1;
+  const int kb0 = gi * KG - bh * n1;
+  const int ow = lane <= KG ? offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + kb0 + lane] : 0;
+  const int lo = __shfl_sync(0xffffffffu, ow, 0);
+  const int hi = __shfl_sync(0xffffffffu, ow, KG);
+  if (lo < 0 || hi < lo || (int64_t)hi > slice_entries) {   // never produced by the transpose
+    if (lane == 0) ucount[gi] = 0;
+    return;
+  }
+  const int32_t* slist = qlist + g.idx_off[1] + (int64_t)bh * slice_entries;
+  int32_t* out = ulist + (int64_t)bh * slice_entries + lo;
+  int* st = stage[warp];
+  const bool staged = hi - lo <= UNION_CAP;
+  if (staged) {
+    for (int e = lane; e < hi - lo; e += 32) st[e] = slist[lo + e];
+    __syncwarp();
+  }
+  // lane j < 8 walks list j
+  int cur = __shfl_sync(0xffffffffu, ow, lane & 7);
+  int end = __shfl_sync(0xffffffffu, ow, (lane & 7) + 1);
+  if (lane >= KG || cur < lo || end < cur || end > hi) cur = end = 0;
+  auto head = [&]() -> int {
+    while (cur < end) {
+      const int a = staged ? st[cur - lo] : slist[cur];
+      if (a >= 0 && a < n1) return a;
+      ++cur;   // an id outside its level: skipped
+    }
+    return 0x7fffffff;
+  };
+  int h = head();
+  int count = 0, val = 0;
+  while (true) {
+    const int q = (int)__reduce_min_sync(0xffffffffu, (unsigned)h);
+    if (q == 0x7fffffff) break;
+    const unsigned msk = __ballot_sync(0xffffffffu, h == q) & 0xffu;
+    if (h == q) {
+      ++cur;
+      h = head();
+    }
+    if (lane == (count & 31)) val = (q << 8) | (int)msk;
+    ++count;
+    if ((count & 31) == 0) out[count - 32 + lane] = val;   // 32 at a time, coalesced
+  }
+  if (lane < (count & 31)) out[(count & ~31) + lane] = val;
+  if (lane == 0) ucount[gi] = count;
+}
+
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const __grid_constant__ Geo g, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo, const float* __restrict__ lse,
-    const float* __restrict__ Dws, const int32_t* __restrict__ offs, const int32_t* __restrict__ qlist,
-    const float* __restrict__ dPK, const float* __restrict__ dPV, __nv_bfloat16* __restrict__ dk,
-    __nv_bfloat16* __restrict__ dv, int* counter, int* err) {
+    const float* __restrict__ Dws, const int32_t* __restrict__ offs, const int32_t* __restrict__ ulist,
+    const int32_t* __restrict__ ucount, const float* __restrict__ dPK, const float* __restrict__ dPV,
+    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,16 +242,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         if (lane == 0) report(err, code);
       }
     };
-    // One chunk of nq query blocks (s.pend_q / s.pend_m) of the group at kbg0:
-    // lane j < nq loads query block j's Q tile, lane 8 + j its dO tile.
-    auto emit = [&](int kbg0, int64_t bh, int nq, int flags) {
+    // One chunk of nq query blocks of the group at kbg0 (lane j < nq holds
+    // member j in pq / pm): lane j loads its Q tile, lane 8 + j its dO tile.
+    auto emit = [&](int kbg0, int64_t bh, int nq, int flags, int pq, int pm) {
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 41);
       if (!ok) return;
       Meta& m = s.meta[slot];
       if (lane < nq) {
-        m.qb[lane] = s.pend_q[lane];
-        m.msk[lane] = s.pend_m[lane];
+        m.qb[lane] = pq;
+        m.msk[lane] = pm;
       }
       __syncwarp();
       uint64_t* bar = &s.full[slot];
@@ -201,8 +267,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       }
       __syncwarp();
       const int j = lane & 7;
+      const int qj = __shfl_sync(0xffffffffu, pq, j);
       if (lane < 16 && j < nq) {
-        const int row = (int)((bh * n1 + s.pend_q[j]) * 16);
+        const int row = (int)((bh * n1 + qj) * 16);
         ChunkSlot& cs = s.slot[slot];
         if (lane < 8)
           ptx::tma_load_2d(cs.q + j * 2048, &tq, 0, row, bar);
@@ -213,83 +280,78 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       ++issued;
     };
 
-    int nxt_l0 = lane == 0 ? atomicAdd(counter, TAKE) : 0;
-    while (ok) {
-      const int g0 = __shfl_sync(0xffffffffu, nxt_l0, 0);
-      if (g0 >= ngroups) break;
-      if (lane == 0) nxt_l0 = atomicAdd(counter, TAKE);   // the take after this one, in flight meanwhile
-      const int ge = g0 + TAKE < ngroups ? g0 + TAKE : ngroups;
-      const int kbf = g0 * KG;                             // first key block taken (global)
-      const int64_t bh = kbf / n1;
-      const int kb0 = (int)(kbf - bh * n1);
-      const int nkb = (ge - g0) * KG;
-      // list starts of the taken key blocks (lane u: block kbf + u; lane nkb: the end)
-      const int ow = lane <= nkb ? offs[g.offs_off[1] + bh * (n1 + 1) + kb0 + lane] : 0;
-      const int32_t* slist = qlist + g.idx_off[1] + bh * slice_entries;   // this slice's CSC entries
-      const int lo = __shfl_sync(0xffffffffu, ow, 0);
-      const int hi = __shfl_sync(0xffffffffu, ow, nkb);
-      const bool staged = lo >= 0 && hi >= lo && hi - lo <= LISTCAP && (int64_t)hi <= slice_entries;
-      if (staged) {
-        for (int e = lane; e < hi - lo; e += 32) s.list[e] = slist[lo + e];
-        __syncwarp();
+    // Group k of this CTA is blockIdx.x + k * gridDim.x.  Lane 0 holds the
+    // start and size of a group's union; all lanes hold its first 64 entries.
+    const int stride = (int)gridDim.x;
+    auto info = [&](int gi, int& lo, int& cnt) {   // issues the loads only
+      lo = cnt = 0;
+      if (gi < ngroups && lane == 0) {
+        const int bh = gi * KG / n1;
+        lo = offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + (gi * KG - bh * n1)];
+        cnt = ucount[gi];
       }
-      for (int gi = g0; gi < ge && ok; ++gi) {
-        const int kbg0 = gi * KG;
-        const int lb = kbg0 - kbf;                         // 0 or 8: the group's first block in the take
-        // the group's K and V: one 16 KB box each
-        {
-          const int ks = (int)(kissued & 1);
-          wait_free(&s.kempty[ks], ((kissued >> 1) & 1) ^ 1, 42);
-          if (!ok) break;
-          if (lane == 0) {
-            ptx::mbar_arrive_expect_tx(&s.kfull[ks], 2u * KG * 2048u);
-            ptx::tma_load_2d(s.key[ks].k, &tk, 0, kbg0 * 16, &s.kfull[ks]);
-            ptx::tma_load_2d(s.key[ks].v, &tv, 0, kbg0 * 16, &s.kfull[ks]);
-          }
-          __syncwarp();
-          ++kissued;
-        }
-        // 8-way merge of the group's sorted lists: lane j < 8 walks list j
-        const int src = lb + (lane & 7);
-        int cur = __shfl_sync(0xffffffffu, ow, src);
-        int end = __shfl_sync(0xffffffffu, ow, src + 1);
-        if (lane >= KG || cur < 0 || end < cur || (int64_t)end > slice_entries) cur = end = 0;
-        auto head = [&]() -> int {
-          while (cur < end) {
-            const int a = staged ? s.list[cur - lo] : slist[cur];
-            if (a >= 0 && a < n1) return a;
-            ++cur;                                         // an id outside its level: skipped
-          }
-          return 0x7fffffff;
-        };
-        int h = head();
-        int pending = 0, emitted = 0;
-        while (ok) {
-          const int q = (int)__reduce_min_sync(0xffffffffu, (unsigned)h);
-          if (q == 0x7fffffff) break;
-          const unsigned msk = __ballot_sync(0xffffffffu, h == q) & 0xffu;
-          if (h == q) {
-            ++cur;
-            h = head();
-          }
-          if (pending == CQ) {
-            emit(kbg0, bh, CQ, emitted == 0 ? kFirst : 0);
-            ++emitted;
-            pending = 0;
-            if (!ok) break;
-          }
-          if (lane == 0) {
-            s.pend_q[pending] = q;
-            s.pend_m[pending] = (int)msk;
-          }
-          __syncwarp();
-          ++pending;
-        }
-        if (ok) emit(kbg0, bh, pending, kLast | (emitted == 0 ? kFirst : 0));
+    };
+    auto entries = [&](int gi, int lo, int cnt, int& e0, int& e1) {
+      e0 = e1 = 0;
+      if (gi < ngroups) {
+        const int32_t* ul = ulist + (int64_t)(gi * KG / n1) * slice_entries + lo;
+        if (lane < cnt) e0 = ul[lane];
+        if (32 + lane < cnt) e1 = ul[32 + lane];
       }
-      __syncwarp();
+    };
+    int gi = (int)blockIdx.x;
+    int lo_c = 0, cnt_c = 0, e0c = 0, e1c = 0;       // group k
+    int lo_n = 0, cnt_n = 0, e0n = 0, e1n = 0;       // group k + 1
+    int lo_nn = 0, cnt_nn = 0;                       // group k + 2 (lane 0)
+    {
+      int a, b;
+      info(gi, a, b);
+      lo_n = __shfl_sync(0xffffffffu, a, 0);
+      cnt_n = __shfl_sync(0xffffffffu, b, 0);
+      entries(gi, lo_n, cnt_n, e0n, e1n);
+      info(gi + stride, lo_nn, cnt_nn);
     }
-    if (ok) {
+    for (; gi < ngroups && ok; gi += stride) {
+      // rotate the prefetch pipeline
+      lo_c = lo_n;
+      cnt_c = cnt_n;
+      e0c = e0n;
+      e1c = e1n;
+      lo_n = __shfl_sync(0xffffffffu, lo_nn, 0);
+      cnt_n = __shfl_sync(0xffffffffu, cnt_nn, 0);
+      entries(gi + stride, lo_n, cnt_n, e0n, e1n);
+      info(gi + 2 * stride, lo_nn, cnt_nn);
+
+      const int kbg0 = gi * KG;
+      const int64_t bh = kbg0 / n1;
+      // the group's K and V: one 16 KB box each
+      {
+        const int ks = (int)(kissued & 1);
+        wait_free(&s.kempty[ks], ((kissued >> 1) & 1) ^ 1, 42);
+        if (!ok) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&s.kfull[ks], 2u * KG * 2048u);
+          ptx::tma_load_2d(s.key[ks].k, &tk, 0, kbg0 * 16, &s.kfull[ks]);
+          ptx::tma_load_2d(s.key[ks].v, &tv, 0, kbg0 * 16, &s.kfull[ks]);
+        }
+        __syncwarp();
+        ++kissued;
+      }
+      const int cnt = cnt_c < 0 ? 0 : cnt_c;
+      const int32_t* ul = ulist + bh * slice_entries + lo_c;
+      const int nchunks = cnt > 0 ? (cnt + CQ - 1) / CQ : 1;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int idx = c * CQ + (lane & 7);
+        const int w0 = __shfl_sync(0xffffffffu, e0c, idx & 31);
+        const int w1 = __shfl_sync(0xffffffffu, e1c, idx & 31);
+        int e = idx < 32 ? w0 : w1;
+        if (idx >= 64 && idx < cnt) e = ul[idx];     // unions longer than 64 (rare)
+        const int nq = cnt - c * CQ < CQ ? cnt - c * CQ : CQ;
+        const int flags = (c == 0 ? kFirst : 0) | (c == nchunks - 1 ? kLast : 0);
+        emit(kbg0, bh, nq > 0 ? nq : 0, flags, e >> 8, e & 0xff);
+      }
+    }
+    if (ok) {   // the end marker: every consumer leaves its loop on it
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 43);
       if (ok && lane == 0) {
@@ -439,12 +501,20 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         tc::fence_after_sync();
         const float l2 = lrow * kLog2e;
 #pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t col = (uint32_t)(half * 64 + j * 16);
-          uint32_t sr[16], pr[16];
-          tc::tmem_ld16(tl + COL_S + col, sr);
-          tc::tmem_ld16(tl + COL_DP + col, pr);
+        for (int jj = 0; jj < 4; jj += 2) {
+          uint32_t sr2[2][16], pr2[2][16];
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint32_t col = (uint32_t)(half * 64 + (jj + t) * 16);
+            tc::tmem_ld16(tl + COL_S + col, sr2[t]);
+            tc::tmem_ld16(tl + COL_DP + col, pr2[t]);
+          }
           tc::tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int j = jj + t;
+          const uint32_t* sr = sr2[t];
+          const uint32_t* pr = pr2[t];
           uint32_t pw[8], dw[8];
           if ((mine >> j) & 1u) {
             float p[16], dsv[16];
@@ -483,6 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
             *reinterpret_cast<uint4*>(s.pbuf + o) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             *reinterpret_cast<uint4*>(s.sbuf + o) = make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
           }
+        }
         }
         tc::fence_before_sync();
         ptx::fence_proxy_async();
@@ -606,12 +677,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
 // Needs n_1 to be a multiple of 16 (checked by the caller): key groups of 8
 // blocks never cross a slice and lie under one level-2 token.
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
-                                  const CUtensorMap& tdo, const float* lse, const float* D, const int32_t* offs,
-                                  const int32_t* qlist, const float* dPK, const float* dPV, void* dk, void* dv,
-                                  int* counter, cudaStream_t s) {
+                                  const CUtensorMap& tdo, const float* lse, const int32_t* offs,
+                                  const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s) {
   CUtensorMap tk, tv;   // one box = one key group (8 blocks, 128 rows)
   cudaError_t e = make_token_map_box(&tk, k, (int64_t)g.BH * g.N, bwdtc::KG * 16);
   if (e == cudaSuccess) e = make_token_map_box(&tv, v, (int64_t)g.BH * g.N, bwdtc::KG * 16);
+  if (e != cudaSuccess) return e;
+  const int ngroups = (int)((int64_t)g.BH * g.n[1] / bwdtc::KG);
+  bwdtc::kv_union_kernel<<<(ngroups + bwdtc::UNION_WARPS - 1) / bwdtc::UNION_WARPS, bwdtc::UNION_WARPS * 32, 0, s>>>(
+      g, offs, qlist, ws.ulist, ws.ucount, ngroups);
+  note_launches(1);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(bwdtc::Smem) + 1024;
   e = cudaFuncSetAttribute(bwdtc::attn_bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -619,9 +695,10 @@ cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, co
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  bwdtc::attn_bwd_kv_tc_kernel<<<sms, bwdtc::THREADS, smem, s>>>(g, tk, tv, tq, tdo, lse, D, offs, qlist, dPK, dPV,
-                                                                  (__nv_bfloat16*)dk, (__nv_bfloat16*)dv, counter,
-                                                                  device_error_word());
+  const int grid = ngroups < sms ? ngroups : sms;
+  bwdtc::attn_bwd_kv_tc_kernel<<<grid, bwdtc::THREADS, smem, s>>>(g, tk, tv, tq, tdo, lse, ws.D, offs, ws.ulist,
+                                                                   ws.ucount, ws.dPK, ws.dPV, (__nv_bfloat16*)dk,
+                                                                   (__nv_bfloat16*)dv, device_error_word());
   note_launches(1);
   return cudaGetLastError();
 }

@@ -495,7 +495,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, ws.D, offs, qlist, ws.dPK, ws.dPV, dk, dv, ws.counter, s);
+  return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, offs, qlist, ws, dk, dv, s);
 }
 
 }  // namespace llsa

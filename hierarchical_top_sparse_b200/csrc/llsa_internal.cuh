@@ -65,6 +65,8 @@ cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, con
                                  const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                  void* dv, void* workspace, cudaStream_t s);
 
+struct BwdWorkspace;
+
 // Tensor-core attention kernels (bf16, d = 64, B = 16).
 bool attn_bwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, const void* v, const void* o,
@@ -72,9 +74,8 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                 void* dv, void* workspace, cudaStream_t s);
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
-                                  const CUtensorMap& tdo, const float* lse, const float* D, const int32_t* offs,
-                                  const int32_t* qlist, const float* dPK, const float* dPV, void* dk, void* dv,
-                                  int* counter, cudaStream_t s);
+                                  const CUtensorMap& tdo, const float* lse, const int32_t* offs,
+                                  const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
 bool attn_fwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
@@ -88,32 +89,44 @@ cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows,
 // Largest candidate count the selection kernel keeps in shared memory.
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
 
-// Workspace of the backward pass: D [BH][N] fp32, then the fp32 level gradients
-// of the pooled K and of the pooled V (each a pyramid), then a work counter.
+// Workspace of the backward pass: D [BH][N] fp32, the fp32 level gradients
+// of the pooled K and of the pooled V (each a pyramid), a work counter, then,
+// for the key-major pass, the union of the query blocks that picked each group
+// of 8 consecutive key blocks (laid out like the level-1 CSC lists, each entry
+// query block << 8 | pick mask) and the size of each union.
 struct BwdWorkspace {
   float* D;
   float* dPK;
   float* dPV;
   int* counter;
+  int32_t* ulist;
+  int32_t* ucount;
   size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counter)
 };
 
-inline size_t bwd_pyr_bytes(const Geo& g) {
-  return ((size_t)g.pyr_off[g.L + 1] * sizeof(float) + 255) & ~(size_t)255;
-}
+inline size_t bwd_round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline size_t bwd_pyr_bytes(const Geo& g) { return bwd_round256((size_t)g.pyr_off[g.L + 1] * sizeof(float)); }
 
 inline size_t bwd_workspace_bytes(const Geo& g) {
-  size_t dsz = (size_t)g.BH * g.N * sizeof(float);
-  dsz = (dsz + 255) & ~(size_t)255;
-  return dsz + 2 * bwd_pyr_bytes(g) + 256;
+  const size_t dsz = bwd_round256((size_t)g.BH * g.N * sizeof(float));
+  const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
+  const size_t csz = bwd_round256(((size_t)g.BH * g.n[1] / 8 + 1) * sizeof(int32_t));
+  return dsz + 2 * bwd_pyr_bytes(g) + 256 + usz + csz;
 }
 
 inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
-  const size_t dsz = ((size_t)g.BH * g.N * sizeof(float) + 255) & ~(size_t)255;
+  const size_t dsz = bwd_round256((size_t)g.BH * g.N * sizeof(float));
   const size_t pyr = bwd_pyr_bytes(g);
+  const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
   char* b = static_cast<char*>(workspace);
-  return BwdWorkspace{reinterpret_cast<float*>(b), reinterpret_cast<float*>(b + dsz),
-                      reinterpret_cast<float*>(b + dsz + pyr), reinterpret_cast<int*>(b + dsz + 2 * pyr),
+  char* after = b + dsz + 2 * pyr + 256;
+  return BwdWorkspace{reinterpret_cast<float*>(b),
+                      reinterpret_cast<float*>(b + dsz),
+                      reinterpret_cast<float*>(b + dsz + pyr),
+                      reinterpret_cast<int*>(b + dsz + 2 * pyr),
+                      reinterpret_cast<int32_t*>(after),
+                      reinterpret_cast<int32_t*>(after + usz),
                       2 * pyr + sizeof(int)};
 }
 
