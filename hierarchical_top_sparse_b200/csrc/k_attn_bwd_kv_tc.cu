@@ -34,9 +34,10 @@
 //     16 KB box each) into one of two key slots, all with TMA;
 //   * warp 13, MMA: a converged warp whose elected lane issues the MMAs and
 //     commits them to mbarriers;
-//   * warps 0-7, softmax: warps w and w + 4 share TMEM lanes 32 (w % 4).. and
-//     take key blocks 0-3 and 4-7 of those query rows;
-//   * warps 8-11, epilogue.
+//   * warps 0-15, softmax: warps w, w + 4, w + 8, w + 12 share TMEM lanes
+//     32 (w % 4).. and take key blocks 2 (w / 4) and 2 (w / 4) + 1 of those
+//     query rows;
+//   * warps 16-19, epilogue.
 // Every hand-off is an mbarrier, every wait is bounded; on a timeout the
 // kernel sets the device error word and stops.
 //
@@ -60,8 +61,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int CQ = 8;               // query blocks per chunk (128 queries)
 constexpr int KG = 8;               // key blocks per group (128 keys)
 constexpr int NSLOT = 3;            // chunk slots
-constexpr int SOFT_WARPS = 8, PRODUCER_WARP = 12, MMA_WARP = 13;   // warps 8-11: epilogue
-constexpr int THREADS = 14 * 32;
+constexpr int SOFT_WARPS = 16, PRODUCER_WARP = 20, MMA_WARP = 21;   // warps 16-19: epilogue
+constexpr int THREADS = 22 * 32;
 constexpr int UNION_WARPS = 8;      // pre-pass: warps per block (one key group each)
 constexpr int UNION_CAP = 512;      // pre-pass: CSC entries of a group staged in shared memory
 constexpr int UPL = 4;              // pooled levels (2..5) whose gradients the epilogue keeps in registers
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         m.qb[lane] = pq;
         m.msk[lane] = pm;
       }
+
       __syncwarp();
       uint64_t* bar = &s.full[slot];
       if (lane == 0) {
@@ -373,7 +375,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     // ============================================================ MMA issue
     // Converged warp, one elected lane issues.  Descriptors are built once and
     // advanced by adding to their start-address field (16-byte units, no
-    // carry: shared addresses are below 256 KB).
+    // carry: shared addresses are below 256 KB).  Software-pipelined: S and
+    // dP of chunk i + 1 are issued as soon as the softmax warps have read
+    // those of chunk i, before dV / dK of chunk i, so that the tensor cores
+    // work while the softmax warps do.
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S, dP: A = Q / dO (K-major), B = K / V (K-major)
     constexpr uint32_t idG = tc::idesc_bf16(64, 128, 1, 1);    // dV^T, dK^T: A = dO / Q (MN-major), B = P / dS (MN-major)
     constexpr uint64_t kSlotStep = sizeof(ChunkSlot) >> 4, kKeyStep = sizeof(KeySlot) >> 4;
@@ -383,31 +388,42 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const uint64_t dv0 = tc::sw128_desc(ptx::smem_u32(s.key[0].v), 16, 1024);
     const uint64_t dp = tc::sw128_desc(ptx::smem_u32(s.pbuf), 16384, 1024);
     const uint64_t dsd = tc::sw128_desc(ptx::smem_u32(s.sbuf), 16384, 1024);
-    uint32_t i = 0, ch = 0, kuse = 0, gacc = 0;
-    bool in_group = false, ok = true;
-    while (ok) {
-      const int slot = (int)(i % NSLOT);
-      if (!ptx::mbar_wait_bounded(&s.full[slot], (i / NSLOT) & 1, kWaitLimitNs)) {
+    bool ok = true;
+    uint32_t seen = 0;        // chunks whose meta words were read (the S side runs one chunk ahead)
+    uint32_t sch = 0;         // chunks with queries whose S / dP were issued
+    uint32_t kseen = 0;       // groups started on the S side
+    // Reads the next chunk's meta and, if it has queries, issues its S / dP.
+    // Returns false on the end marker or a timeout.
+    struct Chunk { int slot, nq, flags, ks; };
+    auto next_s = [&](Chunk& c) -> bool {
+      const int slot = (int)(seen % NSLOT);
+      if (!ptx::mbar_wait_bounded(&s.full[slot], (seen / NSLOT) & 1, kWaitLimitNs)) {
         ok = false;
-        break;
+        return false;
       }
       const Meta& m = s.meta[slot];
-      if (m.kind == kEnd) break;
-      const int nq = m.nq, flags = m.flags;
-      const int ks = (int)(kuse & 1);
-      if (flags & kFirst) {
-        if (!ptx::mbar_wait_bounded(&s.kfull[ks], (kuse >> 1) & 1, kWaitLimitNs)) {
+      if (m.kind == kEnd) return false;
+      c.slot = slot;
+      c.nq = m.nq;
+      c.flags = m.flags;
+      if (c.flags & kFirst) {
+        const int ks = (int)(kseen & 1);
+        if (!ptx::mbar_wait_bounded(&s.kfull[ks], (kseen >> 1) & 1, kWaitLimitNs)) {
           ok = false;
-          break;
+          return false;
         }
+        ++kseen;
       }
-      if (nq > 0) {
-        if (!ptx::mbar_wait_bounded(&s.s_empty, (ch & 1) ^ 1, kWaitLimitNs)) {
+      c.ks = (int)((kseen - 1) & 1);
+      ++seen;
+      if (c.nq > 0) {
+        // the softmax warps have read S / dP of the previous chunk
+        if (!ptx::mbar_wait_bounded(&s.s_empty, (sch & 1) ^ 1, kWaitLimitNs)) {
           ok = false;
-          break;
+          return false;
         }
         tc::fence_after_sync();
-        const uint64_t so = kSlotStep * (uint64_t)slot, ko = kKeyStep * (uint64_t)ks;
+        const uint64_t so = kSlotStep * (uint64_t)slot, ko = kKeyStep * (uint64_t)c.ks;
         if (tc::elect_one()) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {   // K steps of 16 channels: 32 bytes inside the 128-byte rows
@@ -417,7 +433,22 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
           tc::commit(&s.s_full);
         }
         __syncwarp();
-        if (!ptx::mbar_wait_bounded(&s.p_full, ch & 1, kWaitLimitNs)) {
+        ++sch;
+      }
+      return true;
+    };
+
+    uint32_t pch = 0, gacc = 0;   // chunks with queries whose dV / dK were issued; groups accumulated
+    bool in_group = false;
+    Chunk cur;
+    bool have = next_s(cur);
+    while (have && ok) {
+      Chunk nxt;
+      const bool have_next = next_s(nxt);
+      if (!ok) break;
+      // dV / dK of the current chunk
+      if (cur.nq > 0) {
+        if (!ptx::mbar_wait_bounded(&s.p_full, pch & 1, kWaitLimitNs)) {
           ok = false;
           break;
         }
@@ -428,6 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
           }
         }
         tc::fence_after_sync();
+        const uint64_t so = kSlotStep * (uint64_t)cur.slot;
         if (tc::elect_one()) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {   // K steps of 16 queries: two 8-row groups = 2 KB
@@ -435,26 +467,26 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
             tc::mma_bf16(tbase + COL_DK, dq0 + so + 128u * k, dsd + 128u * k, idG, in_group || k > 0);
           }
           tc::commit(&s.p_empty);
-          tc::commit(&s.empty[slot]);
+          tc::commit(&s.empty[cur.slot]);
         }
         __syncwarp();
         in_group = true;
-        ++ch;
+        ++pch;
       } else {
-        if (tc::elect_one()) ptx::mbar_arrive(&s.empty[slot]);
+        if (tc::elect_one()) ptx::mbar_arrive(&s.empty[cur.slot]);
         __syncwarp();
       }
-      if (flags & kLast) {
+      if (cur.flags & kLast) {
         if (tc::elect_one()) {
-          tc::commit(&s.kempty[ks]);   // the group's K and V are free once its MMAs are done
+          tc::commit(&s.kempty[cur.ks]);   // the group's K and V are free once its MMAs are done
           if (in_group) tc::commit(&s.acc_full);
         }
         __syncwarp();
         if (in_group) ++gacc;
         in_group = false;
-        ++kuse;
       }
-      ++i;
+      cur = nxt;
+      have = have_next;
     }
     if (!ok && lane == 0) report(err, 44);
     // every MMA issued here has finished before TMEM is released
@@ -463,15 +495,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     ptx::mbar_wait_bounded(&s.drain, 0, kWaitLimitNs);
   } else if (warp < SOFT_WARPS) {
     // ============================================================ softmax
-    const int sub = warp & 3, half = warp >> 2;
+    const int sub = warp & 3, part = warp >> 2;         // TMEM subpartition; key blocks 2 part, 2 part + 1
     const int row = sub * 32 + lane;                    // query row of the chunk
     const float log2B = log2f((float)g.B);
     const float sc2 = g.scale * kLog2e;
     const bool enrich1 = g.emask & 1u;
     const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
-    // this row's 16-byte chunks in the P / dS operands: half `half`, 8 keys per chunk
-    const uint32_t rbase = (uint32_t)(half * 16384 + (row >> 3) * 1024 + (row & 7) * 128);
     const int r7 = row & 7;
+    // this row's 16-byte chunks of key block kb in the P / dS operands: half kb / 4, chunks 2 (kb % 4) (+1)
+    const uint32_t rbase = (uint32_t)((part >> 1) * 16384 + (row >> 3) * 1024 + (row & 7) * 128);
     uint32_t i = 0, ch = 0;
     while (true) {
       const int slot = (int)(i % NSLOT);
@@ -482,90 +514,93 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       const Meta& m = s.meta[slot];
       if (m.kind == kEnd) break;
       const int nq = m.nq;
+      const int blk = row >> 4;
+      const bool valid = blk < nq;
+      const unsigned mine = valid ? ((unsigned)m.msk[blk] >> (2 * part)) & 3u : 0u;
+      const int qbr = valid ? m.qb[blk] : 0;
+      const int kbg0 = m.kbg0;
+      // only the meta words are needed from the slot (the MMA warp releases the tiles): release it now
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);
       if (nq > 0) {
-        const int blk = row >> 4;
-        const bool valid = blk < nq;
-        const unsigned mine = valid ? ((unsigned)m.msk[blk] >> (4 * half)) & 0xfu : 0u;
-        float lrow = 0.f, Dq = 0.f;
+        float l2 = 0.f, Dq = 0.f;
         if (mine) {   // this row's LSE and D, in flight while the S / dP MMAs run
-          const int bh = m.kbg0 / n1;
-          const int64_t grow = ((int64_t)bh * n1 + m.qb[blk]) * 16 + (row & 15);
-          lrow = lse[grow];
+          const int bh = kbg0 / n1;
+          const int64_t grow = ((int64_t)bh * n1 + qbr) * 16 + (row & 15);
+          l2 = lse[grow] * kLog2e;
           Dq = Dws[grow];
         }
-        if (!ptx::mbar_wait_bounded(&s.s_full, ch & 1, kWaitLimitNs) ||
-            !ptx::mbar_wait_bounded(&s.p_empty, (ch & 1) ^ 1, kWaitLimitNs)) {
+        const unsigned need = __reduce_or_sync(0xffffffffu, mine);   // blocks some row of this warp picked
+        if (!ptx::mbar_wait_bounded(&s.s_full, ch & 1, kWaitLimitNs)) {
           report(err, 46);
           break;
         }
         tc::fence_after_sync();
-        const float l2 = lrow * kLog2e;
-#pragma unroll 1
-        for (int jj = 0; jj < 4; jj += 2) {
-          uint32_t sr2[2][16], pr2[2][16];
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const uint32_t col = (uint32_t)(half * 64 + (jj + t) * 16);
-            tc::tmem_ld16(tl + COL_S + col, sr2[t]);
-            tc::tmem_ld16(tl + COL_DP + col, pr2[t]);
-          }
-          tc::tmem_wait_ld();
+        // P and dS of the row's 2 key blocks, packed bf16 pairs; one block's
+        // S / dP in registers at a time
+        uint32_t pw[2][8], dw[2][8];
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          const int j = jj + t;
-          const uint32_t* sr = sr2[t];
-          const uint32_t* pr = pr2[t];
-          uint32_t pw[8], dw[8];
-          if ((mine >> j) & 1u) {
-            float p[16], dsv[16];
-            float zs = 0.f, dps = 0.f;
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-              const float z = __uint_as_float(sr[n]);
-              const float dpv = __uint_as_float(pr[n]);
-              zs += z;
-              dps += dpv;
-              p[n] = exp2f(fmaf(z, sc2, -l2));
-              dsv[n] = p[n] * (dpv - Dq);
-            }
-            if (enrich1) {
-              const float pc = exp2f(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2) * (1.f / 16.f);
-              const float dsc = pc * (dps * (1.f / 16.f) - Dq);
+          uint32_t sr[16], pr[16];
+          if ((need >> t) & 1u) {
+            const uint32_t col = (uint32_t)((2 * part + t) * 16);
+            tc::tmem_ld16(tl + COL_S + col, sr);
+            tc::tmem_ld16(tl + COL_DP + col, pr);
+            tc::tmem_wait_ld();
+          }
+          if (t == 1) {   // both blocks read: the MMA warp may overwrite S / dP
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s.s_empty);
+          }
+          if ((mine >> t) & 1u) {
+            float pc = 0.f, dsc = 0.f;
+            if (enrich1) {   // the block's pooled level-1 token: mean logit + ln B, mean dP
+              float zs = 0.f, dps = 0.f;
 #pragma unroll
               for (int n = 0; n < 16; ++n) {
-                p[n] += pc;
-                dsv[n] += dsc;
+                zs += __uint_as_float(sr[n]);
+                dps += __uint_as_float(pr[n]);
               }
+              pc = exp2f(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2) * (1.f / 16.f);
+              dsc = pc * (dps * (1.f / 16.f) - Dq);
             }
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
-              pw[n] = ptx::pack_bf16(p[2 * n], p[2 * n + 1]);
-              dw[n] = ptx::pack_bf16(dsv[2 * n], dsv[2 * n + 1]);
+              const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * n]), sc2, -l2));
+              const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * n + 1]), sc2, -l2));
+              const float d0 = fmaf(p0, __uint_as_float(pr[2 * n]) - Dq, dsc);
+              const float d1 = fmaf(p1, __uint_as_float(pr[2 * n + 1]) - Dq, dsc);
+              pw[t][n] = ptx::pack_bf16(p0 + pc, p1 + pc);
+              dw[t][n] = ptx::pack_bf16(d0, d1);
             }
           } else {
 #pragma unroll
-            for (int n = 0; n < 8; ++n) pw[n] = dw[n] = 0u;
+            for (int n = 0; n < 8; ++n) pw[t][n] = dw[t][n] = 0u;
           }
-          // keys 16 j .. 16 j + 15 of this half: 16-byte chunks 2 j and 2 j + 1 of the row
+        }
+        // the operand buffers are free once the previous chunk's dV / dK MMAs are done
+        if (!ptx::mbar_wait_bounded(&s.p_empty, (ch & 1) ^ 1, kWaitLimitNs)) {
+          report(err, 46);
+          break;
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int j = (2 * part + t) & 3;   // block within its half of the keys
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const uint32_t o = rbase + ((uint32_t)((2 * j + c) ^ r7) << 4);
-            *reinterpret_cast<uint4*>(s.pbuf + o) = make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-            *reinterpret_cast<uint4*>(s.sbuf + o) = make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
+            *reinterpret_cast<uint4*>(s.pbuf + o) =
+                make_uint4(pw[t][4 * c], pw[t][4 * c + 1], pw[t][4 * c + 2], pw[t][4 * c + 3]);
+            *reinterpret_cast<uint4*>(s.sbuf + o) =
+                make_uint4(dw[t][4 * c], dw[t][4 * c + 1], dw[t][4 * c + 2], dw[t][4 * c + 3]);
           }
         }
-        }
-        tc::fence_before_sync();
         ptx::fence_proxy_async();
         __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&s.s_empty);
-          ptx::mbar_arrive(&s.p_full);
-        }
+        if (lane == 0) ptx::mbar_arrive(&s.p_full);
         ++ch;
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);   // this warp is done with the slot
       ++i;
     }
   } else {
@@ -586,6 +621,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       if (m.kind == kEnd) break;
       const int kbg0 = m.kbg0, flags = m.flags;
       if (m.nq > 0) group_mma = true;
+      // only the meta words are needed from the slot: release it now
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);
       if (flags & kFirst) {
         // read now, used at the group's last chunk
         const int bh = kbg0 / n1;
@@ -657,8 +695,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         }
         group_mma = false;
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);   // this warp is done with the slot
       ++i;
     }
   }
