@@ -73,6 +73,11 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                 void* dv, void* workspace, cudaStream_t s);
+// Query-major backward on tcgen05: dQ, D = rowsum(dO * O), and the pooled
+// gradients of levels >= 2 (atomics into ws.dPK / ws.dPV, zeroed by the caller).
+cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, const void* v, const void* o,
+                                 const void* dO, const float* lse, const float* pyrK, const float* pyrV,
+                                 const int32_t* idx, const BwdWorkspace& ws, void* dq, cudaStream_t s);
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
                                   const CUtensorMap& tdo, const float* lse, const int32_t* offs,
                                   const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
