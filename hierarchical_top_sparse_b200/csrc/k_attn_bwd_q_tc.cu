@@ -17,27 +17,32 @@
 // accumulated in TMEM over the group's chunks.  The pooled keys of levels >= 2
 // are the same for the token's 256 queries: after the union chunks each group
 // runs one more chunk against them (logit bias ln B^l), adds dS_c Kc to dQ and
-// accumulates their gradients Q^T dS_c and dO^T P_c in TMEM over the token,
-// so each pooled key gets one fp32 atomic per channel and token.
+// accumulates their gradients dS_c^T Q and P_c^T dO in TMEM over the token, so
+// each pooled key gets one fp32 reduction per 4 channels and token.
 //
-// Warp roles, one CTA per SM (22 warps):
+// A pre-pass, q_prep_kernel (one CTA per token), writes what does not need
+// the tensor cores: the unions (each entry (key block << 8) | mask, ascending,
+// in the group's own range of the level-1 index layout), D = rowsum(dO * O)
+// of every query row, and each token's pooled-key tile (bf16 K / V rows in
+// the swizzled operand layout, bias, level, id).
+//
+// Warp roles of the main kernel, one CTA per SM (22 warps):
 //   * warp 20, producer: walks the CTA's tokens (grid stride), loads each
-//     group's Q and dO (one 128-row TMA box each) into one of two group slots
-//     and the K/V tiles of each union chunk (one lane per 2 KB tile) into one
-//     of NSLOT chunk slots, and puts one entry per chunk (and one closing
-//     entry per group) on the chunk ring;
+//     group's Q and dO (one 128-row TMA box each) into one of two group
+//     slots, the token's pooled-key tile (one bulk copy) into one of two
+//     coarse slots, and the K/V tiles of each union chunk (one lane per 2 KB
+//     tile) into one of NSLOT chunk slots, and puts one entry per chunk (and
+//     one closing entry per group) on the chunk ring;
 //   * warp 21, MMA: a converged warp whose elected lane issues every MMA,
 //     the S / dP of chunk i + 1 ahead of the dQ of chunk i;
 //   * warps 0-15, softmax: warps w, w + 4, w + 8, w + 12 share TMEM lanes
 //     32 (w % 4).. and take key blocks 2 (w / 4), 2 (w / 4) + 1 of a chunk;
-//   * warps 16-19, group set-up and epilogue: D = rowsum(dO * O) and LSE of
-//     each group's rows, the token's pooled-key tiles, dQ out of TMEM, and
-//     the pooled-key gradients' atomics.
-// The unions come from a pre-pass, q_union_kernel: one warp per query group
-// merges its 8 sorted pick lists and writes the union in ascending key-block
-// order, each entry (key block << 8) | mask, into the group's own range of the
-// level-1 index layout.  Every hand-off is an mbarrier, every wait is
-// bounded; on a timeout the kernel sets the device error word and stops.
+//     each thread reads its row's LSE and D from global memory at the
+//     group's first entry;
+//   * warps 16-19, epilogue: dQ out of TMEM, and the pooled-key gradients'
+//     reductions.
+// Every hand-off is an mbarrier, every wait is bounded; on a timeout the
+// kernel sets the device error word and stops.
 #include <math.h>
 #include <stddef.h>
 
@@ -56,10 +61,10 @@ constexpr int NSLOT = 3;            // chunk slots
 constexpr int COARSE = 32;          // pooled keys of levels >= 2 per token, at most
 constexpr int SOFT_WARPS = 16, EPI_WARP0 = 16, PRODUCER_WARP = 20, MMA_WARP = 21;
 constexpr int THREADS = 22 * 32;
-constexpr int UNION_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 // S 0-127, dP 128-255, dQ of group slot s at 256 + 64 s, pooled-key
-// gradients dK^T 384-447 and dV^T 448-511 (M = 64: TMEM lanes 0-15 of each quarter)
+// gradients dK 384-447 and dV 448-511 ([pooled key][channel], M = 64: pooled
+// key 16 w + i in TMEM lane 32 w + i)
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_GK = 384, COL_GV = 448;
 enum : int { kEnd = 0, kChunk = 1, kTail = 2 };
 constexpr int kFirst = 1;           // first entry of a group
@@ -75,12 +80,21 @@ struct GroupSlot {
   alignas(1024) unsigned char dO[QG * 2048];
 };
 
-struct CoarseSlot {
-  alignas(1024) unsigned char k[COARSE * 128]; // [32 pooled keys][64] bf16, 128-byte swizzle
-  alignas(1024) unsigned char v[COARSE * 128];
+// A token's pooled keys of levels >= 2, as the pre-pass writes them to the
+// workspace and one bulk copy brings them into shared memory (whose 1024-byte
+// alignment makes the stored swizzle the one the MMA reads).
+struct CoarseTile {
+  unsigned char k[COARSE * 128];               // [32 pooled keys][64] bf16, 128-byte swizzle
+  unsigned char v[COARSE * 128];
   float bias[COARSE];                          // logit bias (log2 domain); -inf: no key
   int level[COARSE];
   int tok[COARSE];                             // pooled token id, -1: none
+};
+static_assert(sizeof(CoarseTile) == kBwdCoarseTileBytes, "the workspace holds one CoarseTile per token");
+static_assert(sizeof(CoarseTile) % 16 == 0, "bulk copies move multiples of 16 bytes");
+
+struct alignas(1024) CoarseSlot {
+  CoarseTile t;
 };
 
 struct Meta {
@@ -98,13 +112,9 @@ struct Smem {
   // The pooled-key chunk uses half 0 for dS_c and half 1 for P_c.
   alignas(1024) unsigned char sbuf[2 * 16384];
   Meta meta[NSLOT];
-  float dsm[2][QG * 16];                       // D of each group slot's rows
-  float lsm[2][QG * 16];                       // LSE (log2 domain) of each group slot's rows
   alignas(8) uint64_t full[NSLOT], empty[NSLOT];
-  uint64_t gfull[2], gempty[2];                // group slots: producer -> MMA / epilogue; MMA + epilogue (4 warps) -> producer
-  uint64_t dready[2];                          // D / LSE of a group slot: epilogue (4 warps) -> softmax
-  uint64_t dfree[2];                           // the softmax warps (16) are done with a group slot's D / LSE
-  uint64_t cfull[2], cempty[2];                // pooled-key tiles: epilogue (4 warps) -> MMA, MMA -> epilogue
+  uint64_t gfull[2], gempty[2];                // group slots: producer -> MMA, MMA -> producer
+  uint64_t cfull[2], cempty[2];                // pooled-key tiles: producer -> MMA, MMA + epilogue (4 warps) -> producer
   uint64_t s_full, s_empty;                    // S / dP in TMEM: MMA -> softmax, softmax (16 warps) -> MMA
   uint64_t p_full, p_empty;                    // dS operand: softmax (16 warps) -> MMA, MMA -> softmax
   uint64_t acc_full[2], acc_empty[2];          // dQ of a group slot: MMA -> epilogue, epilogue (4 warps) -> MMA
@@ -121,17 +131,14 @@ __device__ __forceinline__ void report(int* err, int code) {
   if (err) atomicExch(err, code);
 }
 
-// One warp per query group: the union of the 8 blocks' level-1 pick lists
-// (each sorted ascending), in ascending order, each entry (key block << 8) |
-// mask where bit j says that query block 8 g + j picked the key block.
-// Written at the group's own range of the level-1 index layout (8 K_1 slots);
-// its size in ucount[g].
-__global__ void __launch_bounds__(UNION_WARPS * 32) q_union_kernel(Geo g, const int32_t* __restrict__ idx,
-                                                                   int32_t* __restrict__ ulist,
-                                                                   int32_t* __restrict__ ucount, int ngroups) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gi = blockIdx.x * UNION_WARPS + warp;
-  if (gi >= ngroups) return;
+// One warp: the union of query group gi's 8 level-1 pick lists (each sorted
+// ascending), in ascending order, each entry (key block << 8) | mask where bit
+// j says that query block 8 gi + j picked the key block.  Written at the
+// group's own range of the level-1 index layout (8 K_1 slots); its size in
+// ucount[gi].
+__device__ __forceinline__ void group_union(const Geo& g, const int32_t* __restrict__ idx,
+                                            int32_t* __restrict__ ulist, int32_t* __restrict__ ucount, int gi,
+                                            int lane) {
   const int n1 = g.n[1], K1 = g.Kl[1];
   const int32_t* lists = idx + g.idx_off[1] + (int64_t)gi * QG * K1;   // the group's 8 consecutive lists
   int32_t* out = ulist + (int64_t)gi * QG * K1;
@@ -164,13 +171,92 @@ __global__ void __launch_bounds__(UNION_WARPS * 32) q_union_kernel(Geo g, const 
   if (lane == 0) ucount[gi] = count;
 }
 
+constexpr int PREP_THREADS = 256;
+
+// Pre-pass, one CTA per level-2 token t (query groups 2t, 2t + 1):
+//   * warps 0, 1: the unions of the two groups' pick lists;
+//   * D = rowsum(dO * O) of the token's 256 query rows (8 lanes per row);
+//   * the token's tile of pooled keys of levels >= 2: the lists of level l
+//     belong to the level-(l-1) ancestor of the token's query blocks; each
+//     picked pooled K / V row converted to bf16 at its swizzled place, with
+//     logit bias l ln B (log2 domain), its level and its id.
+__global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32_t* __restrict__ idx,
+                                                              const __nv_bfloat16* __restrict__ o,
+                                                              const __nv_bfloat16* __restrict__ dO,
+                                                              const float* __restrict__ pyrK,
+                                                              const float* __restrict__ pyrV,
+                                                              int32_t* __restrict__ ulist, int32_t* __restrict__ ucount,
+                                                              float* __restrict__ Dws, unsigned char* __restrict__ ctile,
+                                                              int nc) {
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane);
+  const int64_t row0 = (int64_t)t * 2 * QG * 16;
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
+    const int64_t gr = row0 + warp * 32 + it * 4 + (lane >> 3);
+    const uint4 ov = reinterpret_cast<const uint4*>(o + gr * 64)[lane & 7];
+    const uint4 gv = reinterpret_cast<const uint4*>(dO + gr * 64)[lane & 7];
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 a = __bfloat1622float2(o2[e]), b = __bfloat1622float2(g2[e]);
+      acc = fmaf(a.x, b.x, acc);
+      acc = fmaf(a.y, b.y, acc);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if ((lane & 7) == 0) Dws[gr] = acc;
+  }
+  if (nc <= 0) return;
+  const int n1 = g.n[1];
+  const int bh = (2 * t * QG) / n1;
+  const int a0 = 2 * t * QG - bh * n1;                // the token's first query block
+  CoarseTile& ct = *reinterpret_cast<CoarseTile*>(ctile + (size_t)t * sizeof(CoarseTile));
+  const float bias_unit = log2f((float)g.B);          // ln B in the log2 domain
+  for (int e = threadIdx.x; e < COARSE * 16; e += PREP_THREADS) {
+    const int r = e >> 4, chunk = e & 15;
+    int l = 0, tok = -1;
+    if (r < nc) {
+      int rr = r;
+      for (int l2 = 2; l2 <= g.L; ++l2) {
+        if (!((g.emask >> (l2 - 1)) & 1u)) continue;
+        if (rr < g.Kl[l2]) {
+          l = l2;
+          break;
+        }
+        rr -= g.Kl[l2];
+      }
+      const int64_t grp = a0 / g.Bl[l - 1];
+      const int v = idx[g.idx_off[l] + ((int64_t)bh * g.n[l] + grp) * g.Kl[l] + rr];
+      tok = (v >= 0 && v < g.n[l]) ? v : -1;
+    }
+    float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
+    if (tok >= 0) {
+      const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + tok) * 64 + chunk * 4;
+      kv = *reinterpret_cast<const float4*>(pyrK + off);
+      vv = *reinterpret_cast<const float4*>(pyrV + off);
+    }
+    const uint32_t o2 = ptx::sw128(r, chunk * 4);
+    *reinterpret_cast<uint2*>(ct.k + o2) = make_uint2(ptx::pack_bf16(kv.x, kv.y), ptx::pack_bf16(kv.z, kv.w));
+    *reinterpret_cast<uint2*>(ct.v + o2) = make_uint2(ptx::pack_bf16(vv.x, vv.y), ptx::pack_bf16(vv.z, vv.w));
+    if (chunk == 0) {
+      ct.bias[r] = tok >= 0 ? (float)l * bias_unit : -INFINITY;
+      ct.level[r] = l;
+      ct.tok[r] = tok;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     const __grid_constant__ Geo g, const __grid_constant__ CUtensorMap tq128, const __grid_constant__ CUtensorMap tdo128,
-    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, const __nv_bfloat16* __restrict__ o,
-    const __nv_bfloat16* __restrict__ dO, const float* __restrict__ lse, const float* __restrict__ pyrK,
-    const float* __restrict__ pyrV, const int32_t* __restrict__ idx, const int32_t* __restrict__ ulist,
-    const int32_t* __restrict__ ucount, __nv_bfloat16* __restrict__ dq, float* __restrict__ Dws,
-    float* __restrict__ dPK, float* __restrict__ dPV, int* err) {
+    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, const float* __restrict__ lse,
+    const float* __restrict__ Dws, const int32_t* __restrict__ ulist, const int32_t* __restrict__ ucount,
+    const unsigned char* __restrict__ ctile, __nv_bfloat16* __restrict__ dq, float* __restrict__ dPK,
+    float* __restrict__ dPV, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,11 +274,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s.gfull[i], 1);
-      ptx::mbar_init(&s.gempty[i], 1 + 4);
-      ptx::mbar_init(&s.dready[i], 4);
-      ptx::mbar_init(&s.dfree[i], SOFT_WARPS);
-      ptx::mbar_init(&s.cfull[i], 4);
-      ptx::mbar_init(&s.cempty[i], 1);
+      ptx::mbar_init(&s.gempty[i], 1);
+      ptx::mbar_init(&s.cfull[i], 1);
+      ptx::mbar_init(&s.cempty[i], 1 + 4);
       ptx::mbar_init(&s.acc_full[i], 1);
       ptx::mbar_init(&s.acc_empty[i], 4);
     }
@@ -211,9 +295,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     uint4* z = reinterpret_cast<uint4*>(&s.slot[0]);
     const int n16 = (int)(sizeof(ChunkSlot) * NSLOT / 16);
     for (int e = threadIdx.x; e < n16; e += THREADS) z[e] = make_uint4(0u, 0u, 0u, 0u);
-    uint4* zc = reinterpret_cast<uint4*>(&s.crs[0]);
-    const int nc16 = (int)(sizeof(CoarseSlot) * 2 / 16);
-    for (int e = threadIdx.x; e < nc16; e += THREADS) zc[e] = make_uint4(0u, 0u, 0u, 0u);
     ptx::fence_proxy_async();
   }
   if (warp == 0) {
@@ -312,6 +393,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
         __syncwarp();
       };
       load_group(0);
+      if (nc > 0 && ok) {   // the token's pooled-key tile, into coarse slot tk_n % 2
+        const int cs = (int)(tk_n & 1);
+        wait_free(&s.cempty[cs], ((tk_n >> 1) & 1) ^ 1, 52);
+        if (ok && lane == 0) {
+          ptx::mbar_arrive_expect_tx(&s.cfull[cs], (uint32_t)sizeof(CoarseTile));
+          ptx::bulk_load(&s.crs[cs].t, ctile + (size_t)t * sizeof(CoarseTile), (uint32_t)sizeof(CoarseTile),
+                         &s.cfull[cs]);
+        }
+        __syncwarp();
+      }
       for (int gs = 0; gs < 2 && ok; ++gs) {
         const int gi = 2 * t + gs;
         const int64_t bh = (int64_t)gi * QG / n1;
@@ -348,6 +439,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
         ptx::mbar_wait_bounded(&s.full[i % NSLOT], (i / NSLOT) & 1, kWaitLimitNs);
       if (tk_n > 0)
         for (int gs = 0; gs < 2; ++gs) ptx::mbar_wait_bounded(&s.gfull[gs], (tk_n - 1) & 1, kWaitLimitNs);
+      if (nc > 0)   // the last two tokens' pooled-key tiles
+        for (uint32_t k = tk_n > 2 ? tk_n - 2 : 0; k < tk_n; ++k)
+          ptx::mbar_wait_bounded(&s.cfull[k & 1], (k >> 1) & 1, kWaitLimitNs);
     }
     __syncwarp();
   } else if (warp == MMA_WARP) {
@@ -358,17 +452,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S, dP: A = Q / dO (K-major), B = K / V (K-major)
     constexpr uint32_t idSc = tc::idesc_bf16(128, 32, 0, 0);   // the same against the 32 pooled keys
     constexpr uint32_t idQ = tc::idesc_bf16(128, 64, 0, 1);    // dQ += dS K: A = dS (K-major), B = K (MN-major)
-    constexpr uint32_t idG = tc::idesc_bf16(64, 64, 1, 1);     // pooled gradients: A = Q / dO (MN), B = dS_c / P_c (MN)
+    constexpr uint32_t idG = tc::idesc_bf16(64, 64, 1, 1);     // pooled gradients: A = dS_c / P_c (MN), B = Q / dO (MN)
     constexpr uint64_t kSlotStep = sizeof(ChunkSlot) >> 4, kGrpStep = sizeof(GroupSlot) >> 4,
                        kCrsStep = sizeof(CoarseSlot) >> 4;
     const uint64_t dk0 = tc::sw128_desc(ptx::smem_u32(s.slot[0].k), 16, 1024);
     const uint64_t dv0 = tc::sw128_desc(ptx::smem_u32(s.slot[0].v), 16, 1024);
     const uint64_t dq0 = tc::sw128_desc(ptx::smem_u32(s.grp[0].q), 16, 1024);
     const uint64_t do0 = tc::sw128_desc(ptx::smem_u32(s.grp[0].dO), 16, 1024);
-    const uint64_t dck0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].k), 16, 1024);
-    const uint64_t dcv0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].v), 16, 1024);
+    const uint64_t dck0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].t.k), 16, 1024);
+    const uint64_t dcv0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].t.v), 16, 1024);
     const uint64_t dsA = tc::sw128_desc(ptx::smem_u32(s.sbuf), 16, 1024);        // dS as a K-major A operand
-    const uint64_t dsB = tc::sw128_desc(ptx::smem_u32(s.sbuf), 16384, 1024);     // dS_c / P_c as MN-major B operands
+    const uint64_t dsB = tc::sw128_desc(ptx::smem_u32(s.sbuf), 16384, 1024);     // dS_c / P_c as MN-major operands
     bool ok = true;
     // S side (one entry ahead)
     uint32_t seen = 0, sch = 0, tk_s = 0;
@@ -480,10 +574,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
             for (int k = 0; k < 2; ++k)     // dQ += dS_c Kc: 32 pooled keys
               tc::mma_bf16(dqc, dsA + 2u * k, dck0 + co + 128u * k, idQ, dq_started || k > 0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {   // Q^T dS_c, dO^T P_c over the group's 128 queries
+            for (int k = 0; k < 8; ++k) {   // dS_c^T Q, P_c^T dO over the group's 128 queries: [pooled key][channel]
               const bool acc = c.gs == 1 || k > 0;   // the token's second group adds to the first's sums
-              tc::mma_bf16(tbase + COL_GK, dq0 + go + 128u * k, dsB + 128u * k, idG, acc);
-              tc::mma_bf16(tbase + COL_GV, do0 + go + 128u * k, dsB + 1024u + 128u * k, idG, acc);
+              tc::mma_bf16(tbase + COL_GK, dsB + 128u * k, dq0 + go + 128u * k, idG, acc);
+              tc::mma_bf16(tbase + COL_GV, dsB + 1024u + 128u * k, do0 + go + 128u * k, idG, acc);
             }
             tc::commit(&s.p_empty);
           }
@@ -544,6 +638,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     const int r7 = row & 7;
     const uint32_t rrow = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);   // the row inside a 16 KB half
     uint32_t i = 0, ch = 0, tk = 0;
+    // LSE (log2 domain) and D of this thread's row in the current group,
+    // loaded at the group's first entry (their latency hides behind the wait
+    // for its first S)
+    float l2 = 0.f, Dq = 0.f;
     // 16 keys of the row (16-byte chunks 2 j, 2 j + 1 of the row in a 16 KB half); values, not a pointer,
     // so that the words stay in registers
     auto store_row16 = [&](unsigned char* half, int j, uint4 w0, uint4 w1) {
@@ -558,7 +656,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       }
       const Meta& m = s.meta[slot];
       if (m.kind == kEnd) break;
-      const int kind = m.kind, gs = m.gs, nq = m.nq, flags = m.flags;
+      const int kind = m.kind, gs = m.gs, nq = m.nq, flags = m.flags, gi = m.gi;
       unsigned mine = 0;
       if (kind == kChunk) {
 #pragma unroll
@@ -570,15 +668,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       // only the meta words are needed from the slot (the MMA warp releases the tiles): release it now
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);
-      if (flags & kFirst) {   // the group's D and LSE are in shared memory
-        if (!ptx::mbar_wait_bounded(&s.dready[gs], tk & 1, kWaitLimitNs)) {
-          report(err, 56);
-          break;
-        }
+      if (flags & kFirst) {
+        const int64_t grow = (int64_t)gi * QG * 16 + row;
+        l2 = lse[grow] * kLog2e;
+        Dq = Dws[grow];
       }
       const bool has_s = kind == kChunk ? nq > 0 : nc > 0;
       if (has_s) {
-        const float l2 = s.lsm[gs][row], Dq = s.dsm[gs][row];
         if (!ptx::mbar_wait_bounded(&s.s_full, ch & 1, kWaitLimitNs)) {
           report(err, 57);
           break;
@@ -637,6 +733,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
           // pooled keys 16 part .. 16 part + 15 (parts 0, 1; parts 2, 3 write the zero padding),
           // 8 at a time
           uint32_t pw[8], dw[8];
+          // the tile's bias row came by bulk copy: observe its barrier here too
+          if (part < 2 && !ptx::mbar_wait_bounded(&s.cfull[tk & 1], (tk >> 1) & 1, kWaitLimitNs)) {
+            report(err, 56);
+            break;
+          }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t sr[8], pr[8];
@@ -644,7 +745,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
               tc::tmem_ld8(tl + COL_S + 16u * part + 8u * h, sr);
               tc::tmem_ld8(tl + COL_DP + 16u * part + 8u * h, pr);
               tc::tmem_wait_ld();
-              const float* bias = s.crs[tk & 1].bias + 16 * part + 8 * h;
+              const float* bias = s.crs[tk & 1].t.bias + 16 * part + 8 * h;
 #pragma unroll
               for (int n = 0; n < 4; ++n) {
                 float pv[2], dv2[2];
@@ -679,102 +780,21 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
         if (lane == 0) ptx::mbar_arrive(&s.p_full);
         ++ch;
       }
-      if (kind == kTail) {   // the group is done: its D / LSE slot may be refilled
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&s.dfree[gs]);
-        if (gs == 1) ++tk;
-      }
+      if (kind == kTail && gs == 1) ++tk;
       ++i;
     }
   } else {
-    // ============================================================ group set-up and epilogue
-    // Order per token t (k-th of this CTA): dQ of group 0, then the next
-    // token's group-0 D / LSE (its Q / dO have landed once group 0 of t is
-    // done), dQ of group 1, the pooled-key gradients, the next token's group-1
-    // D / LSE; the next token's pooled-key tiles are built first.
+    // ============================================================ epilogue
+    // Per token: dQ of each group out of TMEM, then the pooled-key gradients.
     const int sub = (warp - EPI_WARP0) & 3;             // == warp % 4, the TMEM subpartition this warp may read
     const int row = sub * 32 + lane;                    // query row of a group
     const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
-    const int c16 = sub * 16 + (lane & 15);             // channel of the pooled gradients (lanes 0-15)
-    const float bias_unit = log2f((float)g.B);          // ln B in the log2 domain
     bool ok = true;
     auto fail = [&](int code) {
       report(err, code);
       ok = false;
     };
-    // the token's pooled keys of levels >= 2, as bf16 tiles with their bias
-    auto build_coarse = [&](int t, uint32_t tk) {
-      const int bh = (2 * t * QG) / n1;
-      const int a0 = 2 * t * QG - bh * n1;              // the token's first query block
-      const int ct = (int)(tk & 1);
-      if (!ptx::mbar_wait_bounded(&s.cempty[ct], ((tk >> 1) & 1) ^ 1, kWaitLimitNs)) return fail(59);
-      CoarseSlot& cs = s.crs[ct];
-      for (int e = row; e < COARSE * 16; e += 128) {
-        const int r = e >> 4, chunk = e & 15;
-        int l = 0, tok = -1;
-        if (r < nc) {
-          int rr = r;
-          for (int l2 = 2; l2 <= g.L; ++l2) {
-            if (!((g.emask >> (l2 - 1)) & 1u)) continue;
-            if (rr < g.Kl[l2]) {
-              l = l2;
-              break;
-            }
-            rr -= g.Kl[l2];
-          }
-          const int64_t grp = a0 / g.Bl[l - 1];
-          const int v = idx[g.idx_off[l] + ((int64_t)bh * g.n[l] + grp) * g.Kl[l] + rr];
-          tok = (v >= 0 && v < g.n[l]) ? v : -1;
-        }
-        float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-        if (tok >= 0) {
-          const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + tok) * 64 + chunk * 4;
-          kv = *reinterpret_cast<const float4*>(pyrK + off);
-          vv = *reinterpret_cast<const float4*>(pyrV + off);
-        }
-        const uint32_t o2 = ptx::sw128(r, chunk * 4);
-        *reinterpret_cast<uint2*>(cs.k + o2) = make_uint2(ptx::pack_bf16(kv.x, kv.y), ptx::pack_bf16(kv.z, kv.w));
-        *reinterpret_cast<uint2*>(cs.v + o2) = make_uint2(ptx::pack_bf16(vv.x, vv.y), ptx::pack_bf16(vv.z, vv.w));
-        if (chunk == 0) {
-          cs.bias[r] = tok >= 0 ? (float)l * bias_unit : -INFINITY;
-          cs.level[r] = l;
-          cs.tok[r] = tok;
-        }
-      }
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.cfull[ct]);
-    };
-    // D = rowsum(dO * O) and LSE of a group's rows
-    auto set_up = [&](int t, uint32_t tk, int gs) {
-      if (!ptx::mbar_wait_bounded(&s.dfree[gs], (tk & 1) ^ 1, kWaitLimitNs)) return fail(60);
-      if (!ptx::mbar_wait_bounded(&s.gfull[gs], tk & 1, kWaitLimitNs)) return fail(60);
-      const int64_t grow = (int64_t)(2 * t + gs) * QG * 16 + row;
-      const uint4* orow = reinterpret_cast<const uint4*>(o + grow * 64);
-      float dsum = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 ov = orow[c8];
-        const uint4 gv = *reinterpret_cast<const uint4*>(s.grp[gs].dO + ptx::sw128(row, c8 * 8));
-        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 a = __bfloat1622float2(o2[e]), b = __bfloat1622float2(g2[e]);
-          dsum = fmaf(a.x, b.x, dsum);
-          dsum = fmaf(a.y, b.y, dsum);
-        }
-      }
-      s.dsm[gs][row] = dsum;
-      s.lsm[gs][row] = lse[grow] * kLog2e;
-      Dws[grow] = dsum;
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(&s.dready[gs]);
-        ptx::mbar_arrive(&s.gempty[gs]);   // this warp's reads of dO are done
-      }
-    };
-    // dQ = scale * acc of a group, out of TMEM
+    // dQ = scale * acc of a group
     auto store_dq = [&](int t, uint32_t tk, int gs) {
       if (!ptx::mbar_wait_bounded(&s.acc_full[gs], tk & 1, kWaitLimitNs)) return fail(61);
       tc::fence_after_sync();
@@ -799,53 +819,52 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&s.acc_empty[gs]);
     };
-    // the token's pooled-key gradients: one atomic per (pooled key, channel)
+    // The token's pooled-key gradients: pooled key 16 sub + lane (lanes 0-15)
+    // holds its 64 channels; one 4-wide fp32 reduction per 4 channels.
     auto coarse_grads = [&](int t, uint32_t tk) {
       if (!ptx::mbar_wait_bounded(&s.cacc_full, tk & 1, kWaitLimitNs)) return fail(62);
+      // the tile's ids came by bulk copy: observe its barrier here too
+      if (!ptx::mbar_wait_bounded(&s.cfull[tk & 1], (tk >> 1) & 1, kWaitLimitNs)) return fail(62);
       tc::fence_after_sync();
-      const int bh = (2 * t * QG) / n1;
-      const CoarseSlot& cs = s.crs[tk & 1];
+      const CoarseTile& ct = s.crs[tk & 1].t;
+      if (16 * sub < nc) {
+        const int bh = (2 * t * QG) / n1;
+        const int r = 16 * sub + (lane & 15);
+        const int tok = r < nc ? ct.tok[r] : -1;
+        const int l = ct.level[r];
+        const bool mine = lane < 16 && tok >= 0;
+        const int64_t off = mine ? g.pyr_off[l] + ((int64_t)bh * g.n[l] + tok) * 64 : 0;
 #pragma unroll 1
-      for (int p2 = 0; p2 < 2; ++p2) {
-        uint32_t gk[16], gv[16];
-        tc::tmem_ld16(tl + COL_GK + 16u * p2, gk);
-        tc::tmem_ld16(tl + COL_GV + 16u * p2, gv);
-        tc::tmem_wait_ld();
-        if (lane < 16) {
+        for (int p4 = 0; p4 < 4; ++p4) {
+          uint32_t gk[16], gv[16];
+          tc::tmem_ld16(tl + COL_GK + 16u * p4, gk);
+          tc::tmem_ld16(tl + COL_GV + 16u * p4, gv);
+          tc::tmem_wait_ld();
+          if (mine) {
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            const int r = 16 * p2 + n;
-            const int tok = cs.tok[r];
-            if (r < nc && tok >= 0) {
-              const int l = cs.level[r];
-              const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + tok) * 64 + c16;
-              atomicAdd(dPK + off, __uint_as_float(gk[n]) * g.scale);
-              atomicAdd(dPV + off, __uint_as_float(gv[n]));
+            for (int q = 0; q < 4; ++q) {
+              ptx::red_add_v4(dPK + off + 16 * p4 + 4 * q, __uint_as_float(gk[4 * q]) * g.scale,
+                              __uint_as_float(gk[4 * q + 1]) * g.scale, __uint_as_float(gk[4 * q + 2]) * g.scale,
+                              __uint_as_float(gk[4 * q + 3]) * g.scale);
+              ptx::red_add_v4(dPV + off + 16 * p4 + 4 * q, __uint_as_float(gv[4 * q]), __uint_as_float(gv[4 * q + 1]),
+                              __uint_as_float(gv[4 * q + 2]), __uint_as_float(gv[4 * q + 3]));
             }
           }
         }
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.cacc_empty);
+      if (lane == 0) {
+        ptx::mbar_arrive(&s.cacc_empty);
+        ptx::mbar_arrive(&s.cempty[tk & 1]);   // this warp is done with the tile's ids
+      }
     };
 
-    const int t0 = (int)blockIdx.x;
-    if (t0 < ntokens) {
-      if (nc > 0) build_coarse(t0, 0);
-      if (ok) set_up(t0, 0, 0);
-      if (ok) set_up(t0, 0, 1);
-    }
     uint32_t tk = 0;
-    for (int t = t0; t < ntokens && ok; t += stride, ++tk) {
-      const int tn = t + stride;
-      const bool more = tn < ntokens;
-      if (more && nc > 0) build_coarse(tn, tk + 1);
-      if (ok) store_dq(t, tk, 0);
-      if (ok && more) set_up(tn, tk + 1, 0);
+    for (int t = (int)blockIdx.x; t < ntokens && ok; t += stride, ++tk) {
+      store_dq(t, tk, 0);
       if (ok) store_dq(t, tk, 1);
       if (ok && nc > 0) coarse_grads(t, tk);
-      if (ok && more) set_up(tn, tk + 1, 1);
     }
   }
 
@@ -878,8 +897,11 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   if (e == cudaSuccess) e = make_token_map(&tv, v, rows);
   if (e != cudaSuccess) return e;
   const int ngroups = (int)((int64_t)g.BH * g.n[1] / bwdq::QG);
-  bwdq::q_union_kernel<<<(ngroups + bwdq::UNION_WARPS - 1) / bwdq::UNION_WARPS, bwdq::UNION_WARPS * 32, 0, s>>>(
-      g, idx, ws.ulist, ws.ucount, ngroups);
+  const int ntokens = ngroups / 2;
+  if (ntokens == 0) return cudaSuccess;
+  bwdq::q_prep_kernel<<<ntokens, bwdq::PREP_THREADS, 0, s>>>(g, idx, (const __nv_bfloat16*)o,
+                                                             (const __nv_bfloat16*)dO, pyrK, pyrV, ws.ulist, ws.ucount,
+                                                             ws.D, ws.ctile, nc);
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -889,11 +911,10 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int ntokens = ngroups / 2;
   const int grid = ntokens < sms ? ntokens : sms;
-  bwdq::attn_bwd_q_tc_kernel<<<grid, bwdq::THREADS, smem, s>>>(
-      g, tq128, tdo128, tk, tv, (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, lse, pyrK, pyrV, idx, ws.ulist,
-      ws.ucount, (__nv_bfloat16*)dq, ws.D, ws.dPK, ws.dPV, device_error_word());
+  bwdq::attn_bwd_q_tc_kernel<<<grid, bwdq::THREADS, smem, s>>>(g, tq128, tdo128, tk, tv, lse, ws.D, ws.ulist,
+                                                                ws.ucount, ws.ctile, (__nv_bfloat16*)dq, ws.dPK,
+                                                                ws.dPV, device_error_word());
   note_launches(1);
   return cudaGetLastError();
 }

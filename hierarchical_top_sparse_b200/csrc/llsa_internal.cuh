@@ -95,10 +95,10 @@ cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows,
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
 
 // Workspace of the backward pass: D [BH][N] fp32, the fp32 level gradients
-// of the pooled K and of the pooled V (each a pyramid), a work counter, then,
-// for the key-major pass, the union of the query blocks that picked each group
-// of 8 consecutive key blocks (laid out like the level-1 CSC lists, each entry
-// query block << 8 | pick mask) and the size of each union.
+// of the pooled K and of the pooled V (each a pyramid), a work counter, then
+// the unions of the passes (each entry block << 8 | pick mask, laid out like
+// the level-1 index lists) and the size of each union, then one tile of the
+// pooled keys of levels >= 2 per level-2 token (kBwdCoarseTileBytes each).
 struct BwdWorkspace {
   float* D;
   float* dPK;
@@ -106,8 +106,14 @@ struct BwdWorkspace {
   int* counter;
   int32_t* ulist;
   int32_t* ucount;
+  unsigned char* ctile;
   size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counter)
 };
+
+// A level-2 token's pooled keys of levels >= 2 (at most 32): K and V rows as
+// bf16 [32][64] with the 128-byte swizzle, then per row the logit bias
+// (log2 domain; -inf: no key), the level and the pooled token id (-1: none).
+constexpr size_t kBwdCoarseTileBytes = 2 * 32 * 128 + 3 * 32 * 4;
 
 inline size_t bwd_round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -117,13 +123,15 @@ inline size_t bwd_workspace_bytes(const Geo& g) {
   const size_t dsz = bwd_round256((size_t)g.BH * g.N * sizeof(float));
   const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
   const size_t csz = bwd_round256(((size_t)g.BH * g.n[1] / 8 + 1) * sizeof(int32_t));
-  return dsz + 2 * bwd_pyr_bytes(g) + 256 + usz + csz;
+  const size_t tsz = bwd_round256(((size_t)g.BH * g.n[1] / 16 + 1) * kBwdCoarseTileBytes);
+  return dsz + 2 * bwd_pyr_bytes(g) + 256 + usz + csz + tsz;
 }
 
 inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
   const size_t dsz = bwd_round256((size_t)g.BH * g.N * sizeof(float));
   const size_t pyr = bwd_pyr_bytes(g);
   const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
+  const size_t csz = bwd_round256(((size_t)g.BH * g.n[1] / 8 + 1) * sizeof(int32_t));
   char* b = static_cast<char*>(workspace);
   char* after = b + dsz + 2 * pyr + 256;
   return BwdWorkspace{reinterpret_cast<float*>(b),
@@ -132,6 +140,7 @@ inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
                       reinterpret_cast<int*>(b + dsz + 2 * pyr),
                       reinterpret_cast<int32_t*>(after),
                       reinterpret_cast<int32_t*>(after + usz),
+                      reinterpret_cast<unsigned char*>(after + usz + csz),
                       2 * pyr + sizeof(int)};
 }
 

@@ -160,6 +160,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // Byte offset of element (row, col) of a [rows][64] bf16 tile stored with the
 // 128-byte TMA swizzle (16-byte chunk c of row r sits at chunk c ^ (r & 7));
 // the tile must start on a 1024-byte boundary.
+// Four fp32 additions into global memory by one reduction (no return value);
+// p must be 16-byte aligned.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 __device__ __forceinline__ uint32_t sw128(int row, int col) {
   return (uint32_t)(row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1));
 }
