@@ -56,16 +56,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits for the phase of `parity` to complete, at most `limit_ns` of wall
-// time.  Returns false (and the caller must give up) when the limit passes.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The slow part of a bounded wait, kept out of line and not unrolled: every
+// wait site inlines only its first test, so that the kernels' code stays
+// small enough for the instruction caches.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
   while (true) {
+#pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Waits for the phase of `parity` to complete, at most `limit_ns` of wall
+// time.  Returns false (and the caller must give up) when the limit passes.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, limit_ns);
 }
 
 // Release store / acquire load of a shared-memory word (CTA scope).
@@ -79,15 +88,21 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
   return v;
 }
 
-// Waits until the shared word equals `want`, at most `limit_ns` of wall time.
-__device__ __forceinline__ bool wait_u32_equal(const uint32_t* p, uint32_t want, uint64_t limit_ns) {
-  if (ld_acquire_u32(p) == want) return true;
+static __device__ __noinline__ bool wait_u32_equal_slow(const uint32_t* p, uint32_t want, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
   while (true) {
+#pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (ld_acquire_u32(p) == want) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Waits until the shared word equals `want`, at most `limit_ns` of wall time.
+__device__ __forceinline__ bool wait_u32_equal(const uint32_t* p, uint32_t want, uint64_t limit_ns) {
+  if (ld_acquire_u32(p) == want) return true;
+  return wait_u32_equal_slow(p, want, limit_ns);
 }
 
 // ------------------------------------------------------------------ TMA
