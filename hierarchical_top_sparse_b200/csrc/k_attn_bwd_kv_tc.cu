@@ -14,11 +14,13 @@
 //   pooled level-1 token (mean logit + ln B, mean dP) folded in as P_c / B and
 //   dS_c / B on every key of the block (hierarchical KV enrichment, §四);
 //   blocks it did not pick get zeros;
-//   dV^T += dOc^T P and dK^T += Qc^T dS        (M = 64 channels, N = 128 keys, K = 128 queries)
-// with dV^T and dK^T accumulated in TMEM over the group's chunks.  The 128
-// keys of a group lie under one level-2 token, so they share every pooled key
-// of levels >= 2: the epilogue adds one pooled gradient per channel and level
-// (divided by B^l) and writes dK and dV.
+//   dV += P^T dOc and dK += dS^T Qc            (M = 128 keys, N = 64 channels, K = 128 queries)
+// with dV and dK accumulated in TMEM over the group's chunks, in one of two
+// accumulator buffers, so that the epilogue of a group overlaps the next
+// group's chunks.  The 128 keys of a group lie under one level-2 token, so
+// they share every pooled key of levels >= 2: the epilogue adds one pooled
+// gradient per channel and level (divided by B^l) and writes dK and dV, one
+// key row per thread.
 //
 // Sharing the union's Q/dO tiles among the group's 8 key blocks moves about
 // 2.5x fewer bytes from L2 than gathering them per key block, and N = 128
@@ -26,18 +28,19 @@
 // cost of issuing each MMA; the price is the masked (query block, key block)
 // pairs, computed and discarded.
 //
-// Warp roles, one CTA per SM:
-//   * warp 12, producer: takes the CTA's key groups (grid stride, so that the
+// Warp roles, one CTA per SM (22 warps):
+//   * warp 20, producer: takes the CTA's key groups (grid stride, so that the
 //     CTAs in flight share neighbouring Q/dO tiles in L2), reads each group's
 //     union (prefetched two groups ahead), and loads every chunk (one lane
 //     per 2 KB tile) into one of NSLOT slots and every group's K and V (one
 //     16 KB box each) into one of two key slots, all with TMA;
-//   * warp 13, MMA: a converged warp whose elected lane issues the MMAs and
+//   * warp 21, MMA: a converged warp whose elected lane issues the MMAs and
 //     commits them to mbarriers;
 //   * warps 0-15, softmax: warps w, w + 4, w + 8, w + 12 share TMEM lanes
 //     32 (w % 4).. and take key blocks 2 (w / 4) and 2 (w / 4) + 1 of those
 //     query rows;
-//   * warps 16-19, epilogue.
+//   * warps 16-19, epilogue: walks the CTA's key groups in the same order
+//     and takes each group's accumulators when the MMA warp hands them over.
 // Every hand-off is an mbarrier, every wait is bounded; on a timeout the
 // kernel sets the device error word and stops.
 //
@@ -65,13 +68,13 @@ constexpr int SOFT_WARPS = 16, PRODUCER_WARP = 20, MMA_WARP = 21;   // warps 16-
 constexpr int THREADS = 22 * 32;
 constexpr int UNION_WARPS = 8;      // pre-pass: warps per block (one key group each)
 constexpr int UNION_CAP = 512;      // pre-pass: CSC entries of a group staged in shared memory
-constexpr int UPL = 4;              // pooled levels (2..5) whose gradients the epilogue keeps in registers
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 384;
+// S 0-127, dP 128-255; accumulator buffer b at 256 + 128 b: dV + 0, dK + 64
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
 constexpr int kLast = 1, kFirst = 2;
 enum : int { kEnd = 0, kChunk = 1 };
-// arrivals that free a chunk slot: the MMA thread, each softmax warp, each epilogue warp
-constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS + 4;
+// arrivals that free a chunk slot: the MMA thread and each softmax warp
+constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS;
 
 struct ChunkSlot {
   alignas(1024) unsigned char q[CQ * 2048];    // [128 queries][64] bf16, 128-byte swizzle
@@ -102,8 +105,9 @@ struct Smem {
   uint64_t kfull[2], kempty[2];                // key slots: producer -> MMA, MMA -> producer
   uint64_t s_full, s_empty;                    // S / dP in TMEM: MMA -> softmax, softmax (8 warps) -> MMA
   uint64_t p_full, p_empty;                    // P / dS operands: softmax (8 warps) -> MMA, MMA -> softmax
-  uint64_t acc_full, acc_empty;                // accumulators: MMA -> epilogue, epilogue (4 warps) -> MMA
+  uint64_t acc_full[2], acc_empty[2];          // accumulator buffers: MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t drain;
+  float ukv[2][64];                            // the epilogue's group: pooled-key gradients per channel (K, V)
   uint32_t tmem_base;
 };
 
@@ -202,8 +206,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     ptx::mbar_init(&s.s_empty, SOFT_WARPS);
     ptx::mbar_init(&s.p_full, SOFT_WARPS);
     ptx::mbar_init(&s.p_empty, 1);
-    ptx::mbar_init(&s.acc_full, 1);
-    ptx::mbar_init(&s.acc_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&s.acc_full[i], 1);
+      ptx::mbar_init(&s.acc_empty[i], 4);
+    }
     ptx::mbar_init(&s.drain, 1);
     ptx::fence_mbar_init();
   }
@@ -380,7 +386,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     // those of chunk i, before dV / dK of chunk i, so that the tensor cores
     // work while the softmax warps do.
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S, dP: A = Q / dO (K-major), B = K / V (K-major)
-    constexpr uint32_t idG = tc::idesc_bf16(64, 128, 1, 1);    // dV^T, dK^T: A = dO / Q (MN-major), B = P / dS (MN-major)
+    constexpr uint32_t idG = tc::idesc_bf16(128, 64, 1, 1);    // dV, dK: A = P / dS (MN-major), B = dO / Q (MN-major)
     constexpr uint64_t kSlotStep = sizeof(ChunkSlot) >> 4, kKeyStep = sizeof(KeySlot) >> 4;
     const uint64_t dq0 = tc::sw128_desc(ptx::smem_u32(s.slot[0].q), 16, 1024);
     const uint64_t do0 = tc::sw128_desc(ptx::smem_u32(s.slot[0].dO), 16, 1024);
@@ -438,7 +444,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       return true;
     };
 
-    uint32_t pch = 0, gacc = 0;   // chunks with queries whose dV / dK were issued; groups accumulated
+    uint32_t pch = 0, gcount = 0;   // chunks with queries whose dV / dK were issued; groups closed
     bool in_group = false;
     Chunk cur;
     bool have = next_s(cur);
@@ -452,19 +458,21 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
           ok = false;
           break;
         }
-        if (!in_group) {   // the group's first MMA overwrites the accumulators: wait until they were read
-          if (!ptx::mbar_wait_bounded(&s.acc_empty, (gacc & 1) ^ 1, kWaitLimitNs)) {
+        const uint32_t b = gcount & 1;
+        if (!in_group) {   // the group's first MMA overwrites the buffer: wait until it was read
+          if (!ptx::mbar_wait_bounded(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1, kWaitLimitNs)) {
             ok = false;
             break;
           }
         }
         tc::fence_after_sync();
         const uint64_t so = kSlotStep * (uint64_t)cur.slot;
+        const uint32_t acc = tbase + COL_ACC + 128u * b;
         if (tc::elect_one()) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {   // K steps of 16 queries: two 8-row groups = 2 KB
-            tc::mma_bf16(tbase + COL_DV, do0 + so + 128u * k, dp + 128u * k, idG, in_group || k > 0);
-            tc::mma_bf16(tbase + COL_DK, dq0 + so + 128u * k, dsd + 128u * k, idG, in_group || k > 0);
+            tc::mma_bf16(acc, dp + 128u * k, do0 + so + 128u * k, idG, in_group || k > 0);
+            tc::mma_bf16(acc + 64, dsd + 128u * k, dq0 + so + 128u * k, idG, in_group || k > 0);
           }
           tc::commit(&s.p_empty);
           tc::commit(&s.empty[cur.slot]);
@@ -477,12 +485,19 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         __syncwarp();
       }
       if (cur.flags & kLast) {
+        const uint32_t b = gcount & 1;
+        if (!in_group) {   // no MMA in this group: still hand the buffer over in order
+          if (!ptx::mbar_wait_bounded(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+        }
         if (tc::elect_one()) {
           tc::commit(&s.kempty[cur.ks]);   // the group's K and V are free once its MMAs are done
-          if (in_group) tc::commit(&s.acc_full);
+          tc::commit(&s.acc_full[b]);
         }
         __syncwarp();
-        if (in_group) ++gacc;
+        ++gcount;
         in_group = false;
       }
       cur = nxt;
@@ -605,97 +620,63 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     }
   } else {
     // ============================================================ epilogue
+    // Per key group of this CTA (the producer's order): the pooled-key
+    // gradients per channel, then dK and dV of key row 32 (warp % 4) + lane
+    // out of accumulator buffer k % 2, one 128-byte row each per thread.
     const int sub = warp & 3;
-    const int c = sub * 16 + (lane & 15);               // channel (TMEM lane 32 sub + i <-> row 16 sub + i)
+    const int row = sub * 32 + lane;                    // key of the group (TMEM lane)
+    const int et = threadIdx.x - SOFT_WARPS * 32;       // 0..127
     const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
-    uint32_t i = 0, gacc = 0;
-    bool group_mma = false;
-    float uk = 0.f, uv = 0.f;   // the group's pooled-key gradients on channel c, divided by B^l
-    while (true) {
-      const int slot = (int)(i % NSLOT);
-      if (!ptx::mbar_wait_bounded(&s.full[slot], (i / NSLOT) & 1, kWaitLimitNs)) {
-        report(err, 47);
-        break;
-      }
-      const Meta& m = s.meta[slot];
-      if (m.kind == kEnd) break;
-      const int kbg0 = m.kbg0, flags = m.flags;
-      if (m.nq > 0) group_mma = true;
-      // only the meta words are needed from the slot: release it now
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.empty[slot]);
-      if (flags & kFirst) {
-        // read now, used at the group's last chunk
-        const int bh = kbg0 / n1;
-        const int64_t t0 = (int64_t)(kbg0 - bh * n1) * 16;
-        float kk[UPL], vv[UPL], inv[UPL];
-#pragma unroll
-        for (int j = 0; j < UPL; ++j) {
-          const int l = 2 + j;
-          kk[j] = vv[j] = inv[j] = 0.f;
-          if (l <= g.L && ((g.emask >> (l - 1)) & 1u)) {
-            const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + t0 / g.Bl[l]) * 64 + c;
-            kk[j] = dPK[off];
-            vv[j] = dPV[off];
-            inv[j] = 1.f / (float)g.Bl[l];
-          }
-        }
-        uk = uv = 0.f;
-        for (int l = 2 + UPL; l <= g.L; ++l) {   // deeper hierarchies (rare)
+    uint32_t k = 0;
+    for (int gi = (int)blockIdx.x; gi < ngroups; gi += (int)gridDim.x, ++k) {
+      const int kbg0 = gi * KG;
+      const int bh = kbg0 / n1;
+      const int64_t t0 = (int64_t)(kbg0 - bh * n1) * 16;   // the group's first key within its slice
+      tc::named_sync(1, 128);   // everyone is done with the previous group's values
+      {
+        const int c = et & 63;
+        const float* src = et < 64 ? dPK : dPV;
+        float u = 0.f;
+        for (int l = 2; l <= g.L; ++l) {
           if (!((g.emask >> (l - 1)) & 1u)) continue;
           const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + t0 / g.Bl[l]) * 64 + c;
-          uk = fmaf(dPK[off], 1.f / (float)g.Bl[l], uk);
-          uv = fmaf(dPV[off], 1.f / (float)g.Bl[l], uv);
+          u = fmaf(src[off], 1.f / (float)g.Bl[l], u);
         }
-#pragma unroll
-        for (int j = 0; j < UPL; ++j) {
-          uk = fmaf(kk[j], inv[j], uk);
-          uv = fmaf(vv[j], inv[j], uv);
-        }
+        s.ukv[et >> 6][c] = u;
       }
-      if (flags & kLast) {
-        if (group_mma &&
-            !ptx::mbar_wait_bounded(&s.acc_full, gacc & 1, kWaitLimitNs)) {
-          report(err, 48);
-          break;
-        }
-        tc::fence_after_sync();
-        __nv_bfloat16* pk = dk + (int64_t)kbg0 * 1024 + c;
-        __nv_bfloat16* pv = dv + (int64_t)kbg0 * 1024 + c;
+      tc::named_sync(1, 128);
+      const uint32_t b = k & 1;
+      if (!ptx::mbar_wait_bounded(&s.acc_full[b], (k >> 1) & 1, kWaitLimitNs)) {
+        report(err, 48);
+        break;
+      }
+      tc::fence_after_sync();
+      const bool any = ucount[gi] > 0;                  // else no MMA wrote the buffer
+      const int64_t grow = (int64_t)kbg0 * 16 + row;
 #pragma unroll 1
-        for (int pc = 0; pc < 8; ++pc) {   // 16 keys at a time
-          float av[16], ak[16];
-          if (group_mma) {
-            uint32_t vr[16], kr[16];
-            tc::tmem_ld16(tl + COL_DV + 16u * pc, vr);
-            tc::tmem_ld16(tl + COL_DK + 16u * pc, kr);
-            tc::tmem_wait_ld();
+      for (int h = 0; h < 2; ++h) {                     // dV, then dK
+        uint4* dst = reinterpret_cast<uint4*>((h == 0 ? dv : dk) + grow * 64);
+        const float* u = s.ukv[1 - h];
+        const float f = h == 0 ? 1.f : g.scale;
 #pragma unroll
-            for (int n = 0; n < 16; ++n) {
-              av[n] = __uint_as_float(vr[n]);
-              ak[n] = __uint_as_float(kr[n]) * g.scale;
-            }
-          } else {
+        for (int p4 = 0; p4 < 4; ++p4) {
+          uint32_t r16[16];
+          tc::tmem_ld16(tl + COL_ACC + 128u * b + 64u * (uint32_t)h + 16u * p4, r16);
+          tc::tmem_wait_ld();
+          uint32_t w[8];
 #pragma unroll
-            for (int n = 0; n < 16; ++n) av[n] = ak[n] = 0.f;
+          for (int n = 0; n < 8; ++n) {
+            const float a0 = any ? __uint_as_float(r16[2 * n]) * f : 0.f;
+            const float a1 = any ? __uint_as_float(r16[2 * n + 1]) * f : 0.f;
+            w[n] = ptx::pack_bf16(a0 + u[16 * p4 + 2 * n], a1 + u[16 * p4 + 2 * n + 1]);
           }
-          if (lane < 16) {
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-              pk[(16 * pc + n) * 64] = __float2bfloat16_rn(ak[n] + uk);
-              pv[(16 * pc + n) * 64] = __float2bfloat16_rn(av[n] + uv);
-            }
-          }
+          dst[2 * p4] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[2 * p4 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
-        if (group_mma) {
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&s.acc_empty);
-          ++gacc;
-        }
-        group_mma = false;
       }
-      ++i;
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[b]);
     }
   }
 
