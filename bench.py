@@ -211,12 +211,12 @@ def algorithmic_bytes(stage: str, n, kl, BH: int, N: int, d: int, L: int) -> flo
 
 
 def traffic_record(kernel_stage: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    sources are unchanged since the capture; else None."""
+    """DRAM bytes per launch from the committed ncu summary, if the stage's
+    kernel sources are unchanged since the capture; else None."""
     path = os.path.join(ROOT, "profiles", "traffic_px256.txt")
     if not os.path.exists(path):
         return None
-    digest = sources_digest()
+    digest = sources_digest(kernel_stage)
     for line in open(path):
         f = line.split()
         if len(f) >= 3 and f[0] == kernel_stage and not line.startswith("#"):
@@ -224,12 +224,22 @@ def traffic_record(kernel_stage: str):
     return None
 
 
-def sources_digest() -> str:
+# The sources each stage's kernels are built from (the shared headers included).
+STAGE_SOURCES = {
+    "attn_fwd": ("k_attn_fwd_mma.cu",),
+    "attn_bwd": ("k_attn_bwd.cu", "k_attn_bwd_q_tc.cu", "k_attn_bwd_kv_tc.cu"),
+}
+SHARED_HEADERS = ("llsa_internal.cuh", "ptx.cuh", "tcgen05.cuh", "mma_tiles.cuh")
+
+
+def sources_digest(stage: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hierarchical_top_sparse_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in sorted(STAGE_SOURCES.get(stage, ()) + SHARED_HEADERS):
+        path = os.path.join(csrc, name)
+        if os.path.exists(path):
+            h.update(name.encode())
+            h.update(open(path, "rb").read())
     return h.hexdigest()[:16]
 
 
