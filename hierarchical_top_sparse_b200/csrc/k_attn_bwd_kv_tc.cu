@@ -107,7 +107,6 @@ struct Smem {
   uint64_t p_full, p_empty;                    // P / dS operands: softmax (8 warps) -> MMA, MMA -> softmax
   uint64_t acc_full[2], acc_empty[2];          // accumulator buffers: MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t drain;
-  float ukv[2][64];                            // the epilogue's group: pooled-key gradients per channel (K, V)
   uint32_t tmem_base;
 };
 
@@ -625,26 +624,25 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     // out of accumulator buffer k % 2, one 128-byte row each per thread.
     const int sub = warp & 3;
     const int row = sub * 32 + lane;                    // key of the group (TMEM lane)
-    const int et = threadIdx.x - SOFT_WARPS * 32;       // 0..127
     const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
     uint32_t k = 0;
     for (int gi = (int)blockIdx.x; gi < ngroups; gi += (int)gridDim.x, ++k) {
       const int kbg0 = gi * KG;
       const int bh = kbg0 / n1;
       const int64_t t0 = (int64_t)(kbg0 - bh * n1) * 16;   // the group's first key within its slice
-      tc::named_sync(1, 128);   // everyone is done with the previous group's values
-      {
-        const int c = et & 63;
-        const float* src = et < 64 ? dPK : dPV;
-        float u = 0.f;
-        for (int l = 2; l <= g.L; ++l) {
-          if (!((g.emask >> (l - 1)) & 1u)) continue;
-          const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + t0 / g.Bl[l]) * 64 + c;
-          u = fmaf(src[off], 1.f / (float)g.Bl[l], u);
-        }
-        s.ukv[et >> 6][c] = u;
+      // The group's pooled-key gradients per channel, divided by B^l: lane i
+      // holds channels i and 32 + i (each warp computes its own copy, so
+      // that no barrier joins the epilogue warps).
+      float uk0 = 0.f, uk1 = 0.f, uv0 = 0.f, uv1 = 0.f;
+      for (int l = 2; l <= g.L; ++l) {
+        if (!((g.emask >> (l - 1)) & 1u)) continue;
+        const int64_t off = g.pyr_off[l] + ((int64_t)bh * g.n[l] + t0 / g.Bl[l]) * 64 + lane;
+        const float inv = 1.f / (float)g.Bl[l];
+        uk0 = fmaf(dPK[off], inv, uk0);
+        uk1 = fmaf(dPK[off + 32], inv, uk1);
+        uv0 = fmaf(dPV[off], inv, uv0);
+        uv1 = fmaf(dPV[off + 32], inv, uv1);
       }
-      tc::named_sync(1, 128);
       const uint32_t b = k & 1;
       if (!ptx::mbar_wait_bounded(&s.acc_full[b], (k >> 1) & 1, kWaitLimitNs)) {
         report(err, 48);
@@ -656,7 +654,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {                     // dV, then dK
         uint4* dst = reinterpret_cast<uint4*>((h == 0 ? dv : dk) + grow * 64);
-        const float* u = s.ukv[1 - h];
+        const float u0 = h == 0 ? uv0 : uk0, u1 = h == 0 ? uv1 : uk1;
         const float f = h == 0 ? 1.f : g.scale;
 #pragma unroll
         for (int p4 = 0; p4 < 4; ++p4) {
@@ -666,9 +664,12 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
           uint32_t w[8];
 #pragma unroll
           for (int n = 0; n < 8; ++n) {
+            const int c = 16 * p4 + 2 * n;                // channel of the pair
+            const float b0 = __shfl_sync(0xffffffffu, c < 32 ? u0 : u1, c & 31);
+            const float b1 = __shfl_sync(0xffffffffu, c + 1 < 32 ? u0 : u1, (c + 1) & 31);
             const float a0 = any ? __uint_as_float(r16[2 * n]) * f : 0.f;
             const float a1 = any ? __uint_as_float(r16[2 * n + 1]) * f : 0.f;
-            w[n] = ptx::pack_bf16(a0 + u[16 * p4 + 2 * n], a1 + u[16 * p4 + 2 * n + 1]);
+            w[n] = ptx::pack_bf16(a0 + b0, a1 + b1);
           }
           dst[2 * p4] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[2 * p4 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
