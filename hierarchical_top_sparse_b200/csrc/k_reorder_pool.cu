@@ -120,7 +120,87 @@ static void pool_launch(const Tin* in, float* out, const Geo& g, int64_t total, 
     pool_level_kernel<Tin, 0><<<grid, 256, 0, s>>>(in, out, g.d, g.B, total);
 }
 
+// Levels 1 and 2 in one pass for B = 16, d = 64: one CTA per level-2 token
+// (256 fine rows).  Thread t sums the 16 rows of level-1 token t / 16 on
+// channels 4 (t % 16) .. +3 in row order, divides by B (the same operations
+// as pool_level_kernel), writes it and keeps it in shared memory; then 16
+// threads sum the 16 level-1 values of each channel group in order for the
+// level-2 token.  Lanes 0-15 of a warp read one 128-byte row, lanes 16-31 the
+// next token's.
+template <typename Tin>
+__global__ void __launch_bounds__(256) pool_l12_kernel(const Tin* __restrict__ in, float* __restrict__ p1,
+                                                       float* __restrict__ p2) {
+  constexpr int B = 16, D = 64;
+  __shared__ float4 lvl1[B][D / 4];
+  const int t = threadIdx.x;
+  const int j = t >> 4, c4 = (t & 15) * 4;
+  const int64_t tok2 = blockIdx.x;                   // (slice, level-2 token) flattened
+  const int64_t tok1 = tok2 * B + j;
+  const Tin* src = in + tok1 * B * D + c4;
+  float v[B][4];
+#pragma unroll
+  for (int r = 0; r < B; ++r) load4(src + (int64_t)r * D, v[r]);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int r = 0; r < B; ++r) {
+    acc[0] += v[r][0]; acc[1] += v[r][1]; acc[2] += v[r][2]; acc[3] += v[r][3];
+  }
+  const float4 o = make_float4(acc[0] / B, acc[1] / B, acc[2] / B, acc[3] / B);
+  *reinterpret_cast<float4*>(p1 + tok1 * D + c4) = o;
+  lvl1[j][t & 15] = o;
+  __syncthreads();
+  if (t < D / 4) {
+    float a2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < B; ++r) {
+      const float4 w = lvl1[r][t];
+      a2[0] += w.x; a2[1] += w.y; a2[2] += w.z; a2[3] += w.w;
+    }
+    *reinterpret_cast<float4*>(p2 + tok2 * D + 4 * t) = make_float4(a2[0] / B, a2[1] / B, a2[2] / B, a2[3] / B);
+  }
+}
+
+// Levels 3..L, one CTA per slice: each level from the one below it in global
+// memory (written by this CTA, or by the previous launch for level 2), with
+// the same per-token arithmetic as pool_level_kernel.
+__global__ void __launch_bounds__(256) pool_upper_kernel(float* __restrict__ pyr, Geo g) {
+  const int bh = blockIdx.x;
+  const int c4n = g.d / 4;
+  for (int l = 3; l <= g.L; ++l) {
+    const float* prev = pyr + g.pyr_off[l - 1] + (int64_t)bh * g.n[l - 1] * g.d;
+    float* out = pyr + g.pyr_off[l] + (int64_t)bh * g.n[l] * g.d;
+    const int64_t total = (int64_t)g.n[l] * c4n;
+    for (int64_t e = threadIdx.x; e < total; e += blockDim.x) {
+      const int64_t tok = e / c4n;
+      const int c = (int)(e - tok * c4n) * 4;
+      const float* src = prev + tok * g.B * g.d + c;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int r = 0; r < g.B; ++r) {
+        const float4 w = *reinterpret_cast<const float4*>(src + (int64_t)r * g.d);
+        acc[0] += w.x; acc[1] += w.y; acc[2] += w.z; acc[3] += w.w;
+      }
+      *reinterpret_cast<float4*>(out + tok * g.d + c) =
+          make_float4(acc[0] / g.B, acc[1] / g.B, acc[2] / g.B, acc[3] / g.B);
+    }
+    __syncthreads();   // the level is complete before the next one reads it
+  }
+}
+
 cudaError_t launch_pool(const Geo& g, const void* x, float* pyr, cudaStream_t s) {
+  if (g.B == 16 && g.d == 64 && g.L >= 2) {
+    const unsigned grid = (unsigned)((int64_t)g.BH * g.n[2]);
+    if (g.bf16)
+      pool_l12_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)x, pyr + g.pyr_off[1],
+                                                            pyr + g.pyr_off[2]);
+    else
+      pool_l12_kernel<float><<<grid, 256, 0, s>>>((const float*)x, pyr + g.pyr_off[1], pyr + g.pyr_off[2]);
+    note_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || g.L < 3) return e;
+    pool_upper_kernel<<<g.BH, 256, 0, s>>>(pyr, g);
+    note_launches(1);
+    return cudaGetLastError();
+  }
   for (int l = 1; l <= g.L; ++l) {
     int64_t total = (int64_t)g.BH * g.n[l] * (g.d / 4);
     float* out = pyr + g.pyr_off[l];
