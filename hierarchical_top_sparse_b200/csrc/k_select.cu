@@ -122,7 +122,6 @@ __global__ void __launch_bounds__(selchild::THREADS) select_children_kernel(Geo 
   using namespace selchild;
   __shared__ __align__(16) float ks[NC * LD];
   __shared__ __align__(16) float qs[QB * LD];
-  __shared__ float sc[QB][NC];
   __shared__ int cid[NC];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nl = g.n[l], np = g.n[l + 1];
@@ -134,92 +133,105 @@ __global__ void __launch_bounds__(selchild::THREADS) select_children_kernel(Geo 
   const float* kbase = pyrK + g.pyr_off[l] + (int64_t)bh * nl * 64;
   const float* qbase = pyrQ + g.pyr_off[l] + ((int64_t)bh * nl + (int64_t)par * QB) * 64;
 
-  // candidate ids (position m = pick m / B, child m % B), then the rows
-  if (tid < NC) {
-    int c = -1;
-    if (tid < ncand) {
-      const int pc = plist[tid / QB];
-      c = (pc >= 0 && pc < np) ? pc * QB + tid % QB : -1 - (pc * QB + tid % QB);   // < 0: parent corrupted
-    }
-    cid[tid] = c;
-  }
+  // Candidate m is child m % B of pick m / B.  Every thread resolves the ids of
+  // the rows it copies itself (the parent list is a few cached words), so the
+  // candidate rows and the query rows are fetched in one round.
+  auto cand = [&](int m) -> int {
+    if (m >= ncand) return -1;
+    const int pc = plist[m / QB];
+    return (pc >= 0 && pc < np) ? pc * QB + m % QB : -1 - (pc * QB + m % QB);   // < 0: parent corrupted
+  };
+  if (tid < NC) cid[tid] = cand(tid);
   for (int e = tid; e < QB * 16; e += THREADS) {
     const int r = e >> 4, c4 = (e & 15) * 4;
     *reinterpret_cast<float4*>(&qs[r * LD + c4]) = *reinterpret_cast<const float4*>(qbase + r * 64 + c4);
   }
-  __syncthreads();
   for (int e = tid; e < NC * 16; e += THREADS) {
     const int m = e >> 4, c4 = (e & 15) * 4;
-    const int c = cid[m];
+    const int c = cand(m);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c >= 0) v = *reinterpret_cast<const float4*>(kbase + (int64_t)c * 64 + c4);
     *reinterpret_cast<float4*>(&ks[m * LD + c4]) = v;
   }
   __syncthreads();
 
-  // scores: warp w takes query rows 4w..4w+3, lane the candidates lane + 32 j
-  {
-    float acc[4][4];
+  // scores: warp w takes query rows 4w..4w+3, lane the candidates lane + 32 j;
+  // they stay in registers
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int e = 0; e < 64; e += 4) {
+    float4 qv[4], kv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(&qs[(warp * 4 + i) * LD + e]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kv[j] = *reinterpret_cast<const float4*>(&ks[(lane + 32 * j) * LD + e]);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    for (int e = 0; e < 64; e += 4) {
-      float4 qv[4], kv[4];
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
+        acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
+        acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
+        acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
+      }
+  }
+
+  // top-K_l of the warp's 4 rows, the 4 rows' rounds interleaved so that their
+  // shuffle chains overlap: 64-bit keys (orderable score, then the lower
+  // candidate position wins a tie)
+  uint64_t key[4][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(&qs[(warp * 4 + i) * LD + e]);
+  for (int j = 0; j < 4; ++j) {
+    const int m = lane + 32 * j;
+    const int c = m < ncand ? cid[m] : 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) kv[j] = *reinterpret_cast<const float4*>(&ks[(lane + 32 * j) * LD + e]);
+    for (int i = 0; i < 4; ++i) {
+      if (m >= ncand)
+        key[i][j] = 0;
+      else if (c < 0)
+        key[i][j] = 1ull << 32;          // parent corrupted: the candidate never wins
+      else
+        key[i][j] = ((uint64_t)orderable(acc[i][j]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)m);
+    }
+  }
+  unsigned taken[4] = {0u, 0u, 0u, 0u};
+  for (int k = 0; k < Kl; ++k) {
+    uint64_t best[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+      best[i] = key[i][0];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
-          acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
-          acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
-          acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
-        }
+      for (int j = 1; j < 4; ++j) best[i] = key[i][j] > best[i] ? key[i][j] : best[i];
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sc[warp * 4 + i][lane + 32 * j] = acc[i][j];
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t w = __shfl_xor_sync(0xffffffffu, best[i], o);
+        best[i] = w > best[i] ? w : best[i];
+      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int m = (int)(0xffffffffu - (uint32_t)best[i]);
+      const bool mine = (m & 31) == lane;
+      const int jj = m >> 5;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (mine && j == jj) key[i][j] = 0;
+      if (mine) taken[i] |= 1u << jj;
+    }
   }
-  __syncwarp();
-
-  // top-K_l per query row; rows 4w..4w+3 were scored by this warp
+#pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = warp * 4 + i;
-    uint64_t key[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int m = lane + 32 * j;
-      if (m >= ncand)
-        key[j] = 0;
-      else if (cid[m] < 0)
-        key[j] = 1ull << 32;          // parent corrupted: the candidate never wins
-      else
-        key[j] = ((uint64_t)orderable(sc[r][m]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)m);
-    }
-    unsigned taken = 0;
-    for (int k = 0; k < Kl; ++k) {
-      uint64_t best = key[0];
-#pragma unroll
-      for (int j = 1; j < 4; ++j) best = key[j] > best ? key[j] : best;
-      best = warp_max_u64(best);
-      const int m = (int)(0xffffffffu - (uint32_t)best);
-      if ((m & 31) == lane) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (j == (m >> 5)) key[j] = 0;
-        taken |= 1u << (m >> 5);
-      }
-    }
     int32_t* out = idx + g.idx_off[l] + ((int64_t)bh * nl + (int64_t)par * QB + r) * Kl;
     int written = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const bool t = (taken >> j) & 1u;
+      const bool t = (taken[i] >> j) & 1u;
       const unsigned bal = __ballot_sync(0xffffffffu, t);
       if (t) {
         const int m = lane + 32 * j;
