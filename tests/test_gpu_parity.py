@@ -190,6 +190,7 @@ def test_workload_full_size(cfg, full_slices):
     case = Case(batch=c["batch"], heads=c["heads"], H=c["H"], W=c["W"], L=c["L"], K=c["K"], sigma=c["sigma"])
     run = GpuRun(case, backward=True)
     op = run.op
+    check_pyramids(run)
     check_selection(run)
     check_transpose(run)
     rows = sampled_rows(op.N, 512, 3)
