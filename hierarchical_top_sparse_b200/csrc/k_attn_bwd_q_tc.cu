@@ -14,7 +14,9 @@
 //   token (mean logit + ln B, mean dP) folded in as dS_c / B on each of the
 //   block's 16 keys (hierarchical KV enrichment, §四); other blocks get zeros;
 //   dQ += dS K_c                               (M = 128 queries, N = 64, K = 128 keys)
-// accumulated in TMEM over the group's chunks.  The pooled keys of levels >= 2
+// accumulated in TMEM over the group's chunks, with dS itself written to TMEM
+// by the softmax warps (tcgen05.st) and read from there as the A operand, so
+// that only K_c comes from shared memory.  The pooled keys of levels >= 2
 // are the same for the token's 256 queries: after the union chunks each group
 // runs one more chunk against them (logit bias ln B^l), adds dS_c Kc to dQ and
 // accumulates their gradients dS_c^T Q and P_c^T dO in TMEM over the token, so
@@ -62,10 +64,10 @@ constexpr int COARSE = 32;          // pooled keys of levels >= 2 per token, at 
 constexpr int SOFT_WARPS = 16, EPI_WARP0 = 16, PRODUCER_WARP = 20, MMA_WARP = 21;
 constexpr int THREADS = 22 * 32;
 constexpr uint32_t TMEM_COLS = 512;
-// S 0-127, dP 128-255, dQ of group slot s at 256 + 64 s, pooled-key
-// gradients dK 384-447 and dV 448-511 ([pooled key][channel], M = 64: pooled
-// key 16 w + i in TMEM lane 32 w + i)
-constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_GK = 384, COL_GV = 448;
+// S 0-127, dP 128-255, dQ 256-319, dS of a chunk 320-383 (bf16 pairs: the A
+// operand of dQ += dS K), pooled-key gradients dK 384-447 and dV 448-511
+// ([pooled key][channel], M = 64: pooled key 16 w + i in TMEM lane 32 w + i)
+constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_DS = 320, COL_GK = 384, COL_GV = 448;
 enum : int { kEnd = 0, kChunk = 1, kTail = 2 };
 constexpr int kFirst = 1;           // first entry of a group
 constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS;   // a chunk slot is freed by the MMA thread and every softmax warp
@@ -117,7 +119,7 @@ struct Smem {
   uint64_t cfull[2], cempty[2];                // pooled-key tiles: producer -> MMA, MMA + epilogue (4 warps) -> producer
   uint64_t s_full, s_empty;                    // S / dP in TMEM: MMA -> softmax, softmax (16 warps) -> MMA
   uint64_t p_full, p_empty;                    // dS operand: softmax (16 warps) -> MMA, MMA -> softmax
-  uint64_t acc_full[2], acc_empty[2];          // dQ of a group slot: MMA -> epilogue, epilogue (4 warps) -> MMA
+  uint64_t acc_full, acc_empty;                // dQ of a group (phase = the CTA's group count): MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t cacc_full, cacc_empty;              // pooled-key gradients: MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t drain;
   uint32_t tmem_base;
@@ -277,13 +279,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       ptx::mbar_init(&s.gempty[i], 1);
       ptx::mbar_init(&s.cfull[i], 1);
       ptx::mbar_init(&s.cempty[i], 1 + 4);
-      ptx::mbar_init(&s.acc_full[i], 1);
-      ptx::mbar_init(&s.acc_empty[i], 4);
     }
     ptx::mbar_init(&s.s_full, 1);
     ptx::mbar_init(&s.s_empty, SOFT_WARPS);
     ptx::mbar_init(&s.p_full, SOFT_WARPS);
     ptx::mbar_init(&s.p_empty, 1);
+    ptx::mbar_init(&s.acc_full, 1);
+    ptx::mbar_init(&s.acc_empty, 4);
     ptx::mbar_init(&s.cacc_full, 1);
     ptx::mbar_init(&s.cacc_empty, 4);
     ptx::mbar_init(&s.drain, 1);
@@ -536,15 +538,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     bool dq_started = false;
     auto finish = [&](const Entry& c) {
       const uint64_t go = kGrpStep * (uint64_t)c.gs;
-      const uint32_t dqc = tbase + COL_DQ + 64u * (uint32_t)c.gs;
+      const uint32_t dqc = tbase + COL_DQ;
       const bool has_s = c.kind == kChunk ? c.nq > 0 : nc > 0;
       if (has_s) {
         if (!ptx::mbar_wait_bounded(&s.p_full, pch & 1, kWaitLimitNs)) {
           ok = false;
           return;
         }
-        if (!dq_started) {   // the group's first dQ MMA overwrites the accumulator: wait until it was read
-          if (!ptx::mbar_wait_bounded(&s.acc_empty[c.gs], (c.tk & 1) ^ 1, kWaitLimitNs)) {
+        if (!dq_started) {   // the group's first dQ MMA overwrites the accumulator: wait until the last group's was read
+          if (!ptx::mbar_wait_bounded(&s.acc_empty, (uint32_t)(c.gs ^ 1), kWaitLimitNs)) {
             ok = false;
             return;
           }
@@ -560,10 +562,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
           const uint64_t so = kSlotStep * (uint64_t)c.slot;
           if (tc::elect_one()) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {   // 16 keys per K step: A 32 bytes (64-key halves 16 KB apart), B 2 KB
-              const uint64_t ao = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);
-              tc::mma_bf16(dqc, dsA + ao, dk0 + so + 128u * k, idQ, dq_started || k > 0);
-            }
+            for (int k = 0; k < 8; ++k)     // 16 keys per K step: A 8 TMEM columns, B 2 KB
+              tc::mma_bf16_ta(dqc, tbase + COL_DS + 8u * k, dk0 + so + 128u * k, idQ, dq_started || k > 0);
             tc::commit(&s.p_empty);
             tc::commit(&s.empty[c.slot]);
           }
@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       }
       if (c.kind == kTail) {
         if (!dq_started) {   // no dQ MMA in this group: still hand the (unused) accumulator over in order
-          if (!ptx::mbar_wait_bounded(&s.acc_empty[c.gs], (c.tk & 1) ^ 1, kWaitLimitNs)) {
+          if (!ptx::mbar_wait_bounded(&s.acc_empty, (uint32_t)(c.gs ^ 1), kWaitLimitNs)) {
             ok = false;
             return;
           }
@@ -596,7 +596,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
         if (tc::elect_one()) {
           if (!has_s) ptx::mbar_arrive(&s.empty[c.slot]);   // nothing of this entry in flight
           else tc::commit(&s.empty[c.slot]);
-          tc::commit(&s.acc_full[c.gs]);     // the group's dQ is complete
+          tc::commit(&s.acc_full);           // the group's dQ is complete
           tc::commit(&s.gempty[c.gs]);       // its Q and dO are free
           if (c.gs == 1 && nc > 0) {
             tc::commit(&s.cacc_full);        // the token's pooled-key gradients are complete
@@ -721,14 +721,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
               for (int n = 0; n < 8; ++n) dw[t][n] = 0u;
             }
           }
+          // dQ(i - 1) has read the previous dS from TMEM
           if (!ptx::mbar_wait_bounded(&s.p_empty, (ch & 1) ^ 1, kWaitLimitNs)) {
             report(err, 58);
             break;
           }
+          tc::fence_after_sync();
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
-            store_row16(s.sbuf + (part >> 1) * 16384, (2 * part + t) & 3, make_uint4(dw[t][0], dw[t][1], dw[t][2], dw[t][3]),
-                        make_uint4(dw[t][4], dw[t][5], dw[t][6], dw[t][7]));
+          for (int t = 0; t < 2; ++t) tc::tmem_st8(tl + COL_DS + 8u * (uint32_t)(2 * part + t), dw[t]);
+          tc::tmem_wait_st();
         } else {
           // pooled keys 16 part .. 16 part + 15 (parts 0, 1; parts 2, 3 write the zero padding),
           // 8 at a time
@@ -775,7 +776,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
           store_row16(s.sbuf, part, make_uint4(dw[0], dw[1], dw[2], dw[3]), make_uint4(dw[4], dw[5], dw[6], dw[7]));
           store_row16(s.sbuf + 16384, part, make_uint4(pw[0], pw[1], pw[2], pw[3]), make_uint4(pw[4], pw[5], pw[6], pw[7]));
         }
-        ptx::fence_proxy_async();
+        ptx::fence_proxy_async();   // the tail's operands are in shared memory
+        tc::fence_before_sync();    // a chunk's dS is in TMEM
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&s.p_full);
         ++ch;
@@ -796,7 +798,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     };
     // dQ = scale * acc of a group
     auto store_dq = [&](int t, uint32_t tk, int gs) {
-      if (!ptx::mbar_wait_bounded(&s.acc_full[gs], tk & 1, kWaitLimitNs)) return fail(61);
+      // group 2 tk + gs of this CTA: that phase's parity is gs
+      if (!ptx::mbar_wait_bounded(&s.acc_full, (uint32_t)gs, kWaitLimitNs)) return fail(61);
       tc::fence_after_sync();
       const int gi = 2 * t + gs;
       const bool any = nc > 0 || ucount[gi] > 0;        // else no MMA wrote the accumulator: dQ = 0
@@ -805,7 +808,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
 #pragma unroll
       for (int p4 = 0; p4 < 4; ++p4) {
         uint32_t r16[16];
-        tc::tmem_ld16(tl + COL_DQ + 64u * (uint32_t)gs + 16u * p4, r16);
+        tc::tmem_ld16(tl + COL_DQ + 16u * p4, r16);
         tc::tmem_wait_ld();
         uint32_t w[8];
 #pragma unroll
@@ -817,7 +820,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.acc_empty[gs]);
+      if (lane == 0) ptx::mbar_arrive(&s.acc_empty);
     };
     // The token's pooled-key gradients: pooled key 16 sub + lane (lanes 0-15)
     // holds its 64 channels; one 4-wide fp32 reduction per 4 channels.
