@@ -138,11 +138,21 @@ __device__ __forceinline__ void report(int* err, int code) {
 // j says that query block 8 gi + j picked the key block.  Written at the
 // group's own range of the level-1 index layout (8 K_1 slots); its size in
 // ucount[gi].
+// The lists are first staged in `stage` (UNION_STAGE words) when they fit,
+// so that the merge loop reads shared memory rather than a chain of
+// dependent global loads.
+constexpr int UNION_STAGE = 512;
 __device__ __forceinline__ void group_union(const Geo& g, const int32_t* __restrict__ idx,
                                             int32_t* __restrict__ ulist, int32_t* __restrict__ ucount, int gi,
-                                            int lane) {
+                                            int lane, int* stage) {
   const int n1 = g.n[1], K1 = g.Kl[1];
-  const int32_t* lists = idx + g.idx_off[1] + (int64_t)gi * QG * K1;   // the group's 8 consecutive lists
+  const int32_t* glists = idx + g.idx_off[1] + (int64_t)gi * QG * K1;   // the group's 8 consecutive lists
+  const bool staged = QG * K1 <= UNION_STAGE;
+  if (staged) {
+    for (int e = lane; e < QG * K1; e += 32) stage[e] = glists[e];
+    __syncwarp();
+  }
+  const int32_t* lists = staged ? stage : glists;
   int32_t* out = ulist + (int64_t)gi * QG * K1;
   // lane j < 8 walks list j
   int cur = lane < QG ? lane * K1 : 0;
@@ -190,9 +200,10 @@ __global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32
                                                               int32_t* __restrict__ ulist, int32_t* __restrict__ ucount,
                                                               float* __restrict__ Dws, unsigned char* __restrict__ ctile,
                                                               int nc) {
+  __shared__ int stage[2][UNION_STAGE];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane);
+  if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane, stage[warp]);
   const int64_t row0 = (int64_t)t * 2 * QG * 16;
 #pragma unroll 2
   for (int it = 0; it < 8; ++it) {
