@@ -135,8 +135,8 @@ __global__ void scatter_kernel(Geo g, TransposeArgs a) {
   }
 }
 
-constexpr int kSortWarps = 4;
-constexpr int kBitmapWords = 2048;   // 65536 query ids per window
+constexpr int kSortWarps = 8;
+constexpr int kBitmapWords = 256;    // 8192 query ids per window (a small array keeps 8 blocks per SM resident)
 
 // One warp per (level, slice, key): writes the key's query ids ascending.
 __global__ void __launch_bounds__(kSortWarps * 32) sort_kernel(Geo g, TransposeArgs a) {
