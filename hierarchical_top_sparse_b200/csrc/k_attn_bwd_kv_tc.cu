@@ -576,13 +576,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
                 zs += __uint_as_float(sr[n]);
                 dps += __uint_as_float(pr[n]);
               }
-              pc = exp2f(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2) * (1.f / 16.f);
+              pc = ptx::ex2(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2) * (1.f / 16.f);
               dsc = pc * (dps * (1.f / 16.f) - Dq);
             }
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
-              const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * n]), sc2, -l2));
-              const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * n + 1]), sc2, -l2));
+              const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * n]), sc2, -l2));
+              const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * n + 1]), sc2, -l2));
               const float d0 = fmaf(p0, __uint_as_float(pr[2 * n]) - Dq, dsc);
               const float d1 = fmaf(p1, __uint_as_float(pr[2 * n + 1]) - Dq, dsc);
               pw[t][n] = ptx::pack_bf16(p0 + pc, p1 + pc);

@@ -717,13 +717,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
                   zs += __uint_as_float(sr[n]);
                   dps += __uint_as_float(pr[n]);
                 }
-                const float pc = exp2f(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2);
+                const float pc = ptx::ex2(fmaf(zs * (1.f / 16.f), sc2, log2B) - l2);
                 dsc = pc * (dps * (1.f / 16.f) - Dq) * (1.f / 16.f);
               }
 #pragma unroll
               for (int n = 0; n < 8; ++n) {
-                const float p0 = exp2f(fmaf(__uint_as_float(sr[2 * n]), sc2, -l2));
-                const float p1 = exp2f(fmaf(__uint_as_float(sr[2 * n + 1]), sc2, -l2));
+                const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * n]), sc2, -l2));
+                const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * n + 1]), sc2, -l2));
                 dw[t][n] = ptx::pack_bf16(fmaf(p0, __uint_as_float(pr[2 * n]) - Dq, dsc),
                                           fmaf(p1, __uint_as_float(pr[2 * n + 1]) - Dq, dsc));
               }
@@ -764,7 +764,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                   const float b = bias[2 * n + e];
-                  const float p = b == -INFINITY ? 0.f : exp2f(fmaf(__uint_as_float(sr[2 * n + e]), sc2, b) - l2);
+                  const float p = b == -INFINITY ? 0.f : ptx::ex2(fmaf(__uint_as_float(sr[2 * n + e]), sc2, b) - l2);
                   pv[e] = p;
                   dv2[e] = p * (__uint_as_float(pr[2 * n + e]) - Dq);
                 }

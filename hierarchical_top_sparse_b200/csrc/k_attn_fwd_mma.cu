@@ -94,7 +94,7 @@ struct RowState {
 };
 
 __device__ __forceinline__ void rescale(RowState& st, float mn0, float mn1) {
-  const float a0 = exp2f(st.m[0] - mn0), a1 = exp2f(st.m[1] - mn1);
+  const float a0 = ptx::ex2(st.m[0] - mn0), a1 = ptx::ex2(st.m[1] - mn1);
   st.m[0] = mn0;
   st.m[1] = mn1;
   st.l[0] *= a0;
@@ -203,7 +203,7 @@ __device__ __forceinline__ void fine_batch(RowState& st, const uint32_t (*qa)[4]
     if (i < npend) {
       float sh0 = 0.f, sh1 = 0.f;
       if (enrich1) {
-        const float pc0 = exp2f(zc[i][0] - mn0), pc1 = exp2f(zc[i][1] - mn1);
+        const float pc0 = ptx::ex2(zc[i][0] - mn0), pc1 = ptx::ex2(zc[i][1] - mn1);
         if (tq4 == 0) {
           st.l[0] += pc0;
           st.l[1] += pc1;
@@ -214,10 +214,10 @@ __device__ __forceinline__ void fine_batch(RowState& st, const uint32_t (*qa)[4]
       float p[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        p[j][0] = exp2f(z[i][j][0] - mn0);
-        p[j][1] = exp2f(z[i][j][1] - mn0);
-        p[j][2] = exp2f(z[i][j][2] - mn1);
-        p[j][3] = exp2f(z[i][j][3] - mn1);
+        p[j][0] = ptx::ex2(z[i][j][0] - mn0);
+        p[j][1] = ptx::ex2(z[i][j][1] - mn0);
+        p[j][2] = ptx::ex2(z[i][j][2] - mn1);
+        p[j][3] = ptx::ex2(z[i][j][3] - mn1);
         st.l[0] += p[j][0] + p[j][1];
         st.l[1] += p[j][2] + p[j][3];
       }
@@ -553,10 +553,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
       float p[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        p[j][0] = exp2f(z[j][0] - mn0);
-        p[j][1] = exp2f(z[j][1] - mn0);
-        p[j][2] = exp2f(z[j][2] - mn1);
-        p[j][3] = exp2f(z[j][3] - mn1);
+        p[j][0] = ptx::ex2(z[j][0] - mn0);
+        p[j][1] = ptx::ex2(z[j][1] - mn0);
+        p[j][2] = ptx::ex2(z[j][2] - mn1);
+        p[j][3] = ptx::ex2(z[j][3] - mn1);
         st.l[0] += p[j][0] + p[j][1];
         st.l[1] += p[j][2] + p[j][3];
       }

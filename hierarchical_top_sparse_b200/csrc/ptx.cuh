@@ -175,6 +175,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // Byte offset of element (row, col) of a [rows][64] bf16 tile stored with the
 // 128-byte TMA swizzle (16-byte chunk c of row r sits at chunk c ^ (r & 7));
 // the tile must start on a 1024-byte boundary.
+// 2^x by the PTX approximate base-2 exponential (ex2.approx.ftz.f32: a few ulp
+// of relative error, results below 2^-126 flushed to zero, 2^-inf = 0).  The
+// softmax weights it produces are rounded to bf16 right after.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Four fp32 additions into global memory by one reduction (no return value);
 // p must be 16-byte aligned.
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
