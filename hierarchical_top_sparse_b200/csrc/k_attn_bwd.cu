@@ -50,7 +50,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   BwdWorkspace ws = carve_bwd_workspace(g, workspace);
   e = cudaMemsetAsync(ws.dPK, 0, ws.zero_bytes, s);   // pooled-key sums and the work counter
   if (e != cudaSuccess) return e;
-  e = launch_attn_bwd_q_tc(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, ws, dq, s);
+  e = launch_attn_bwd_q_tc(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, ws, dq, s);
   if (e != cudaSuccess) return e;
   return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, offs, qlist, ws, dk, dv, s);
 }

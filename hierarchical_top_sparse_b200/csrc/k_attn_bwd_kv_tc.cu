@@ -44,11 +44,11 @@
 // Every hand-off is an mbarrier, every wait is bounded; on a timeout the
 // kernel sets the device error word and stops.
 //
-// The unions come from a pre-pass, kv_union_kernel: one warp per key group
-// merges the group's 8 sorted level-1 CSC lists and writes the union in
-// ascending query-block order, each entry (query block << 8) | pick mask,
-// into the group's own range of the CSC layout (a union is never longer than
-// the lists it merges).
+// The unions come from the query-major pre-pass (q_prep_kernel): one warp per
+// key group merges the group's 8 sorted level-1 CSC lists and writes the
+// union in ascending query-block order, each entry (query block << 8) | pick
+// mask, into the group's own range of the CSC layout (a union is never longer
+// than the lists it merges).
 #include <math.h>
 #include <stddef.h>
 
@@ -66,8 +66,6 @@ constexpr int KG = 8;               // key blocks per group (128 keys)
 constexpr int NSLOT = 3;            // chunk slots
 constexpr int SOFT_WARPS = 16, PRODUCER_WARP = 20, MMA_WARP = 21;   // warps 16-19: epilogue
 constexpr int THREADS = 22 * 32;
-constexpr int UNION_WARPS = 8;      // pre-pass: warps per block (one key group each)
-constexpr int UNION_CAP = 512;      // pre-pass: CSC entries of a group staged in shared memory
 constexpr uint32_t TMEM_COLS = 512;
 // S 0-127, dP 128-255; accumulator buffer b at 256 + 128 b: dV + 0, dK + 64
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
@@ -116,67 +114,6 @@ static_assert(sizeof(ChunkSlot) % 1024 == 0 && sizeof(KeySlot) % 1024 == 0,
 
 __device__ __forceinline__ void report(int* err, int code) {
   if (err) atomicExch(err, code);
-}
-
-// One warp per key group: the union of the 8 blocks' level-1 CSC lists (each
-// sorted ascending), in ascending order, each entry (query block << 8) | mask
-// where bit j says that the query block picked key block 8 g + j.  Written at
-// the group's own CSC range [offs(8 g), offs(8 g) + size); size in ucount[g].
-__global__ void __launch_bounds__(UNION_WARPS * 32) kv_union_kernel(Geo g, const int32_t* __restrict__ offs,
-                                                                    const int32_t* __restrict__ qlist,
-                                                                    int32_t* __restrict__ ulist,
-                                                                    int32_t* __restrict__ ucount, int ngroups) {
-  __shared__ int stage[UNION_WARPS][UNION_CAP];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gi = blockIdx.x * UNION_WARPS + warp;
-  if (gi >= ngroups) return;
-  const int n1 = g.n[1];
-  const int64_t slice_entries = (int64_t)n1 * g.Kl[1];
-  const int bh = gi * KG / n1;
-  const int kb0 = gi * KG - bh * n1;
-  const int ow = lane <= KG ? offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + kb0 + lane] : 0;
-  const int lo = __shfl_sync(0xffffffffu, ow, 0);
-  const int hi = __shfl_sync(0xffffffffu, ow, KG);
-  if (lo < 0 || hi < lo || (int64_t)hi > slice_entries) {   // never produced by the transpose
-    if (lane == 0) ucount[gi] = 0;
-    return;
-  }
-  const int32_t* slist = qlist + g.idx_off[1] + (int64_t)bh * slice_entries;
-  int32_t* out = ulist + (int64_t)bh * slice_entries + lo;
-  int* st = stage[warp];
-  const bool staged = hi - lo <= UNION_CAP;
-  if (staged) {
-    for (int e = lane; e < hi - lo; e += 32) st[e] = slist[lo + e];
-    __syncwarp();
-  }
-  // lane j < 8 walks list j
-  int cur = __shfl_sync(0xffffffffu, ow, lane & 7);
-  int end = __shfl_sync(0xffffffffu, ow, (lane & 7) + 1);
-  if (lane >= KG || cur < lo || end < cur || end > hi) cur = end = 0;
-  auto head = [&]() -> int {
-    while (cur < end) {
-      const int a = staged ? st[cur - lo] : slist[cur];
-      if (a >= 0 && a < n1) return a;
-      ++cur;   // an id outside its level: skipped
-    }
-    return 0x7fffffff;
-  };
-  int h = head();
-  int count = 0, val = 0;
-  while (true) {
-    const int q = (int)__reduce_min_sync(0xffffffffu, (unsigned)h);
-    if (q == 0x7fffffff) break;
-    const unsigned msk = __ballot_sync(0xffffffffu, h == q) & 0xffu;
-    if (h == q) {
-      ++cur;
-      h = head();
-    }
-    if (lane == (count & 31)) val = (q << 8) | (int)msk;
-    ++count;
-    if ((count & 31) == 0) out[count - 32 + lane] = val;   // 32 at a time, coalesced
-  }
-  if (lane < (count & 31)) out[(count & ~31) + lane] = val;
-  if (lane == 0) ucount[gi] = count;
 }
 
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
@@ -702,11 +639,6 @@ cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, co
   if (e == cudaSuccess) e = make_token_map_box(&tv, v, (int64_t)g.BH * g.N, bwdtc::KG * 16);
   if (e != cudaSuccess) return e;
   const int ngroups = (int)((int64_t)g.BH * g.n[1] / bwdtc::KG);
-  bwdtc::kv_union_kernel<<<(ngroups + bwdtc::UNION_WARPS - 1) / bwdtc::UNION_WARPS, bwdtc::UNION_WARPS * 32, 0, s>>>(
-      g, offs, qlist, ws.ulist, ws.ucount, ngroups);
-  note_launches(1);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const size_t smem = sizeof(bwdtc::Smem) + 1024;
   e = cudaFuncSetAttribute(bwdtc::attn_bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -714,8 +646,8 @@ cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, co
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = ngroups < sms ? ngroups : sms;
-  bwdtc::attn_bwd_kv_tc_kernel<<<grid, bwdtc::THREADS, smem, s>>>(g, tk, tv, tq, tdo, lse, ws.D, offs, ws.ulist,
-                                                                   ws.ucount, ws.dPK, ws.dPV, (__nv_bfloat16*)dk,
+  bwdtc::attn_bwd_kv_tc_kernel<<<grid, bwdtc::THREADS, smem, s>>>(g, tk, tv, tq, tdo, lse, ws.D, offs, ws.ulist_kv,
+                                                                   ws.ucount_kv, ws.dPK, ws.dPV, (__nv_bfloat16*)dk,
                                                                    (__nv_bfloat16*)dv, device_error_word());
   note_launches(1);
   return cudaGetLastError();

@@ -183,10 +183,70 @@ __device__ __forceinline__ void group_union(const Geo& g, const int32_t* __restr
   if (lane == 0) ucount[gi] = count;
 }
 
+// One warp: the union of key group gi's 8 level-1 CSC lists (each sorted
+// ascending), in ascending order, each entry (query block << 8) | mask where
+// bit j says that the query block picked key block 8 gi + j.  Written at the
+// group's own CSC range [offs(8 gi), offs(8 gi) + size) of ulist; its size in
+// ucount[gi].  For the key-major pass.
+__device__ __forceinline__ void key_group_union(const Geo& g, const int32_t* __restrict__ offs,
+                                                const int32_t* __restrict__ qlist, int32_t* __restrict__ ulist,
+                                                int32_t* __restrict__ ucount, int gi, int lane, int* stage) {
+  constexpr int KG = 8;
+  const int n1 = g.n[1];
+  const int64_t slice_entries = (int64_t)n1 * g.Kl[1];
+  const int bh = gi * KG / n1;
+  const int kb0 = gi * KG - bh * n1;
+  const int ow = lane <= KG ? offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + kb0 + lane] : 0;
+  const int lo = __shfl_sync(0xffffffffu, ow, 0);
+  const int hi = __shfl_sync(0xffffffffu, ow, KG);
+  if (lo < 0 || hi < lo || (int64_t)hi > slice_entries) {   // never produced by the transpose
+    if (lane == 0) ucount[gi] = 0;
+    return;
+  }
+  const int32_t* slist = qlist + g.idx_off[1] + (int64_t)bh * slice_entries;
+  int32_t* out = ulist + (int64_t)bh * slice_entries + lo;
+  const bool staged = hi - lo <= UNION_STAGE;
+  if (staged) {
+    for (int e = lane; e < hi - lo; e += 32) stage[e] = slist[lo + e];
+    __syncwarp();
+  }
+  // lane j < 8 walks list j
+  int cur = __shfl_sync(0xffffffffu, ow, lane & 7);
+  int end = __shfl_sync(0xffffffffu, ow, (lane & 7) + 1);
+  if (lane >= KG || cur < lo || end < cur || end > hi) cur = end = 0;
+  auto head = [&]() -> int {
+    while (cur < end) {
+      const int a = staged ? stage[cur - lo] : slist[cur];
+      if (a >= 0 && a < n1) return a;
+      ++cur;   // an id outside its level: skipped
+    }
+    return 0x7fffffff;
+  };
+  int h = head();
+  int count = 0, val = 0;
+  while (true) {
+    const int q = (int)__reduce_min_sync(0xffffffffu, (unsigned)h);
+    if (q == 0x7fffffff) break;
+    const unsigned msk = __ballot_sync(0xffffffffu, h == q) & 0xffu;
+    if (h == q) {
+      ++cur;
+      h = head();
+    }
+    if (lane == (count & 31)) val = (q << 8) | (int)msk;
+    ++count;
+    if ((count & 31) == 0) out[count - 32 + lane] = val;   // 32 at a time, coalesced
+  }
+  if (lane < (count & 31)) out[(count & ~31) + lane] = val;
+  if (lane == 0) ucount[gi] = count;
+}
+
 constexpr int PREP_THREADS = 256;
 
-// Pre-pass, one CTA per level-2 token t (query groups 2t, 2t + 1):
-//   * warps 0, 1: the unions of the two groups' pick lists;
+// Pre-pass, one CTA per level-2 token t (query groups 2t, 2t + 1; key groups
+// 2t, 2t + 1 are the same 16 blocks as keys):
+//   * warps 0, 1: the unions of the two query groups' pick lists;
+//   * warps 2, 3: the unions of the two key groups' CSC lists (for the
+//     key-major pass);
 //   * D = rowsum(dO * O) of the token's 256 query rows (8 lanes per row);
 //   * the token's tile of pooled keys of levels >= 2: the lists of level l
 //     belong to the level-(l-1) ancestor of the token's query blocks; each
@@ -197,13 +257,18 @@ __global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32
                                                               const __nv_bfloat16* __restrict__ dO,
                                                               const float* __restrict__ pyrK,
                                                               const float* __restrict__ pyrV,
+                                                              const int32_t* __restrict__ offs,
+                                                              const int32_t* __restrict__ qlist,
                                                               int32_t* __restrict__ ulist, int32_t* __restrict__ ucount,
+                                                              int32_t* __restrict__ ulist_kv,
+                                                              int32_t* __restrict__ ucount_kv,
                                                               float* __restrict__ Dws, unsigned char* __restrict__ ctile,
                                                               int nc) {
-  __shared__ int stage[2][UNION_STAGE];
+  __shared__ int stage[4][UNION_STAGE];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane, stage[warp]);
+  else if (warp < 4) key_group_union(g, offs, qlist, ulist_kv, ucount_kv, 2 * t + warp - 2, lane, stage[warp]);
   const int64_t row0 = (int64_t)t * 2 * QG * 16;
 #pragma unroll 2
   for (int it = 0; it < 8; ++it) {
@@ -897,7 +962,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
 // levels >= 2; anything else returns cudaErrorInvalidValue before a launch.
 cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, const void* v, const void* o,
                                  const void* dO, const float* lse, const float* pyrK, const float* pyrV,
-                                 const int32_t* idx, const BwdWorkspace& ws, void* dq, cudaStream_t s) {
+                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist,
+                                 const BwdWorkspace& ws, void* dq, cudaStream_t s) {
   int nc = 0;
   for (int l = 2; l <= g.L; ++l)
     if ((g.emask >> (l - 1)) & 1u) nc += g.Kl[l];
@@ -914,8 +980,9 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   const int ntokens = ngroups / 2;
   if (ntokens == 0) return cudaSuccess;
   bwdq::q_prep_kernel<<<ntokens, bwdq::PREP_THREADS, 0, s>>>(g, idx, (const __nv_bfloat16*)o,
-                                                             (const __nv_bfloat16*)dO, pyrK, pyrV, ws.ulist, ws.ucount,
-                                                             ws.D, ws.ctile, nc);
+                                                             (const __nv_bfloat16*)dO, pyrK, pyrV, offs, qlist,
+                                                             ws.ulist, ws.ucount, ws.ulist_kv, ws.ucount_kv, ws.D,
+                                                             ws.ctile, nc);
   note_launches(1);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

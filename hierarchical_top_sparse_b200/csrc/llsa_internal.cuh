@@ -77,7 +77,8 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
 // gradients of levels >= 2 (atomics into ws.dPK / ws.dPV, zeroed by the caller).
 cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, const void* v, const void* o,
                                  const void* dO, const float* lse, const float* pyrK, const float* pyrV,
-                                 const int32_t* idx, const BwdWorkspace& ws, void* dq, cudaStream_t s);
+                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist,
+                                 const BwdWorkspace& ws, void* dq, cudaStream_t s);
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
                                   const CUtensorMap& tdo, const float* lse, const int32_t* offs,
                                   const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
@@ -96,9 +97,10 @@ constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
 
 // Workspace of the backward pass: D [BH][N] fp32, the fp32 level gradients
 // of the pooled K and of the pooled V (each a pyramid), a work counter, then
-// the unions of the passes (each entry block << 8 | pick mask, laid out like
-// the level-1 index lists) and the size of each union, then one tile of the
-// pooled keys of levels >= 2 per level-2 token (kBwdCoarseTileBytes each).
+// the query groups' unions (each entry block << 8 | pick mask, laid out like
+// the level-1 index lists) and their sizes, one tile of the pooled keys of
+// levels >= 2 per level-2 token (kBwdCoarseTileBytes each), then the key
+// groups' unions (laid out like the level-1 CSC lists) and their sizes.
 struct BwdWorkspace {
   float* D;
   float* dPK;
@@ -107,6 +109,8 @@ struct BwdWorkspace {
   int32_t* ulist;
   int32_t* ucount;
   unsigned char* ctile;
+  int32_t* ulist_kv;
+  int32_t* ucount_kv;
   size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counter)
 };
 
@@ -124,7 +128,7 @@ inline size_t bwd_workspace_bytes(const Geo& g) {
   const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
   const size_t csz = bwd_round256(((size_t)g.BH * g.n[1] / 8 + 1) * sizeof(int32_t));
   const size_t tsz = bwd_round256(((size_t)g.BH * g.n[1] / 16 + 1) * kBwdCoarseTileBytes);
-  return dsz + 2 * bwd_pyr_bytes(g) + 256 + usz + csz + tsz;
+  return dsz + 2 * bwd_pyr_bytes(g) + 256 + 2 * (usz + csz) + tsz;
 }
 
 inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
@@ -132,8 +136,10 @@ inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
   const size_t pyr = bwd_pyr_bytes(g);
   const size_t usz = bwd_round256((size_t)g.BH * g.n[1] * g.Kl[1] * sizeof(int32_t));
   const size_t csz = bwd_round256(((size_t)g.BH * g.n[1] / 8 + 1) * sizeof(int32_t));
+  const size_t tsz = bwd_round256(((size_t)g.BH * g.n[1] / 16 + 1) * kBwdCoarseTileBytes);
   char* b = static_cast<char*>(workspace);
   char* after = b + dsz + 2 * pyr + 256;
+  char* kv = after + usz + csz + tsz;
   return BwdWorkspace{reinterpret_cast<float*>(b),
                       reinterpret_cast<float*>(b + dsz),
                       reinterpret_cast<float*>(b + dsz + pyr),
@@ -141,6 +147,8 @@ inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
                       reinterpret_cast<int32_t*>(after),
                       reinterpret_cast<int32_t*>(after + usz),
                       reinterpret_cast<unsigned char*>(after + usz + csz),
+                      reinterpret_cast<int32_t*>(kv),
+                      reinterpret_cast<int32_t*>(kv + usz),
                       2 * pyr + sizeof(int)};
 }
 
