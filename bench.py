@@ -229,7 +229,7 @@ STAGE_SOURCES = {
     "attn_fwd": ("k_attn_fwd_mma.cu",),
     "attn_bwd": ("k_attn_bwd.cu", "k_attn_bwd_q_tc.cu", "k_attn_bwd_kv_tc.cu"),
 }
-SHARED_HEADERS = ("llsa_internal.cuh", "ptx.cuh", "tcgen05.cuh", "mma_tiles.cuh")
+SHARED_HEADERS = ("llsa_internal.cuh", "ptx.cuh", "tcgen05.cuh")
 
 
 def sources_digest(stage: str) -> str:

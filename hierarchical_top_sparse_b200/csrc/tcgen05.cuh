@@ -141,27 +141,5 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// Named barrier over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Named barrier that also returns the AND of `pred` over the `count` threads,
-// so that a decision taken after a bounded wait is the same in every thread.
-__device__ __forceinline__ bool named_and(int id, int count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n"
-      ".reg .pred p, q;\n"
-      "setp.ne.u32 p, %1, 0;\n"
-      "bar.red.and.pred q, %2, %3, p;\n"
-      "selp.u32 %0, 1, 0, q;\n"
-      "}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
-}
-
 }  // namespace tc
 }  // namespace llsa
