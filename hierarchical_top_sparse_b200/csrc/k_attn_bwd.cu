@@ -52,7 +52,7 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
   if (e != cudaSuccess) return e;
   e = launch_attn_bwd_q_tc(g, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, ws, dq, s);
   if (e != cudaSuccess) return e;
-  return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, offs, qlist, ws, dk, dv, s);
+  return launch_attn_bwd_kv_tc(g, k, v, tq, tdo, lse, offs, ws, dk, dv, s);
 }
 
 }  // namespace llsa

@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
 // blocks never cross a slice and lie under one level-2 token.
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
                                   const CUtensorMap& tdo, const float* lse, const int32_t* offs,
-                                  const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s) {
+                                  const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s) {
   CUtensorMap tk, tv;   // one box = one key group (8 blocks, 128 rows)
   cudaError_t e = make_token_map_box(&tk, k, (int64_t)g.BH * g.N, bwdtc::KG * 16);
   if (e == cudaSuccess) e = make_token_map_box(&tv, v, (int64_t)g.BH * g.N, bwdtc::KG * 16);

@@ -81,7 +81,7 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
                                  const BwdWorkspace& ws, void* dq, cudaStream_t s);
 cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
                                   const CUtensorMap& tdo, const float* lse, const int32_t* offs,
-                                  const int32_t* qlist, const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
+                                  const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
 bool attn_fwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
