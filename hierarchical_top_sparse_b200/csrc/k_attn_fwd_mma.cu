@@ -37,7 +37,8 @@ constexpr int MAXPICK = 256;     // G * K_1, at most
 constexpr int MAXWORDS = 2048;   // union bitmap: level-1 blocks per slice, at most 65536
 constexpr int BATCH = 2;         // picked blocks per softmax batch (9 warps: 168 registers at most)
 constexpr int TMA_WARP = G;
-constexpr int THREADS = (G + 1) * 32;
+constexpr int UNION_WARP = G + 1;
+constexpr int THREADS = (G + 2) * 32;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: a wait this long means something broke
 
 struct Smem {
@@ -58,6 +59,7 @@ struct Smem {
   uint64_t empty[SLOTS];
   uint64_t qfull[NBUF];    // query tiles landed (TMA) and the union list written
   uint64_t qempty[NBUF];   // the group's consumers are done with the buffer
+  uint64_t ufull[NBUF];    // the union list is written: union warp -> TMA warp
   uint64_t csync;          // consumer-wide barrier around the pooled-key tile
   int abort_flag;
 };
@@ -258,6 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     for (int b = 0; b < NBUF; ++b) {
       ptx::mbar_init(&s.qfull[b], 2);     // the TMA bytes' arrival and the union list's arrival
       ptx::mbar_init(&s.qempty[b], G);
+      ptx::mbar_init(&s.ufull[b], 1);
     }
     ptx::mbar_init(&s.csync, G * 32);
     s.abort_flag = 0;
@@ -289,13 +292,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     return 2 * ((int)blockIdx.x + (it >> 1) * (int)gridDim.x) + (it & 1);
   };
 
-  if (warp == TMA_WARP) {
-    // ----------------------------------------- union of the picks, TMA loads
-    if (lane == 0) {
-      ptx::prefetch_tmap(&tq);
-      ptx::prefetch_tmap(&tk);
-      ptx::prefetch_tmap(&tv);
-    }
+  if (warp == UNION_WARP) {
+    // ----------------------------------------- union of the picks (a group ahead of the TMA warp)
     const int np = G * K1;
     const bool small = np <= 64;
     auto pick_ptr = [&](int gi) {
@@ -314,14 +312,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     for (int gi = group_of(0); gi < ngroups; gi = group_of(++it)) {
       const int b = it % NBUF;
       const uint32_t use = (uint32_t)(it / NBUF);
-      const int bh = gi / groups_per_slice;
-      const int a0 = (gi - bh * groups_per_slice) * G;
       if (lane == 0 && !ptx::mbar_wait_bounded(&s.qempty[b], (use & 1) ^ 1, kWaitLimitNs)) give_up(s, err, 1);
       __syncwarp();
       if (aborted(s)) break;
-      if (lane == 0) ptx::mbar_arrive_expect_tx(&s.qfull[b], G * 2048);
-      __syncwarp();
-      if (lane < G) ptx::tma_load_2d(s.q[b][lane], &tq, 0, bh * g.N + (a0 + lane) * 16, &s.qfull[b]);
       int nu = 0;
       int o0 = 0x7fffffff, o1 = 0x7fffffff;   // picks 2*lane, 2*lane+1 in pick order (small case)
       if (small) {
@@ -410,7 +403,40 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
         }
       }
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.qfull[b]);     // union list and pick positions visible
+      if (lane == 0) {
+        ptx::mbar_arrive(&s.qfull[b]);     // union list and pick positions visible to the consumers
+        ptx::mbar_arrive(&s.ufull[b]);     // and to the TMA warp
+      }
+      ring_pos += (uint32_t)nu;
+      __syncwarp();
+    }
+    return;
+  }
+
+  if (warp == TMA_WARP) {
+    // ----------------------------------------- query tiles and the union's K/V blocks, TMA
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tq);
+      ptx::prefetch_tmap(&tk);
+      ptx::prefetch_tmap(&tv);
+    }
+    uint32_t ring_pos = 0;
+    int it = 0;
+    for (int gi = group_of(0); gi < ngroups; gi = group_of(++it)) {
+      const int b = it % NBUF;
+      const uint32_t use = (uint32_t)(it / NBUF);
+      const int bh = gi / groups_per_slice;
+      const int a0 = (gi - bh * groups_per_slice) * G;
+      if (lane == 0 && !ptx::mbar_wait_bounded(&s.qempty[b], (use & 1) ^ 1, kWaitLimitNs)) give_up(s, err, 1);
+      __syncwarp();
+      if (aborted(s)) break;
+      if (lane == 0) ptx::mbar_arrive_expect_tx(&s.qfull[b], G * 2048);
+      __syncwarp();
+      if (lane < G) ptx::tma_load_2d(s.q[b][lane], &tq, 0, bh * g.N + (a0 + lane) * 16, &s.qfull[b]);
+      if (lane == 0 && !ptx::mbar_wait_bounded(&s.ufull[b], use & 1, kWaitLimitNs)) give_up(s, err, 1);
+      __syncwarp();
+      if (aborted(s)) break;
+      const int nu = s.ucount[b];
       // one lane per ring position
       bool ok = true;
       for (int u0 = 0; u0 < nu; u0 += 32) {
