@@ -5,16 +5,19 @@
 // level-2 parent).  The 8 blocks pick their K_1 key blocks among the same
 // candidates, so their picks overlap; the group loads the UNION of its picks
 // once.  One persistent CTA per SM, each on a contiguous range of groups:
-//   * a TMA warp sorts and deduplicates the group's picks and streams the
-//     union's K/V blocks (2 KB each) with TMA 2-D tile loads (128-byte
-//     swizzle) through a ring of slots guarded by mbarriers, one lane per
-//     slot;
-//   * 8 consumer warps, one per query block, convert the group's pooled keys
-//     of levels >= 2 (shared by all 128 queries) to bf16 once per level-2
-//     parent, then walk the union in order and feed the blocks they picked,
-//     two at a time, through warp-level MMA (m16n8k16, bf16 in, fp32
-//     accumulate): exactly K_1 * B fine keys plus the pooled keys per query,
-//     no masked work, the online softmax in registers.
+//   * a union warp sorts and deduplicates the group's picks, a group ahead;
+//   * a TMA warp streams the union's K/V blocks (2 KB each) with TMA 2-D
+//     tile loads (128-byte swizzle) through a ring of slots guarded by
+//     mbarriers, one lane per slot;
+//   * 16 consumer warps, two per query block, convert the group's pooled
+//     keys of levels >= 2 (shared by all 128 queries) to bf16 once per
+//     level-2 parent; each warp then takes every other one of its block's
+//     picks (and half of the pooled keys), walks the union in order and
+//     feeds them through warp-level MMA (m16n8k16, bf16 in, fp32 accumulate)
+//     with the online softmax in registers: exactly K_1 * B fine keys plus
+//     the pooled keys per query, no masked work.  The second warp of a block
+//     hands its running max, sum and O (as bf16) to the first through shared
+//     memory, which merges them and writes O and LSE.
 // A pooled level-1 token is the mean of the 16 keys of the block it stands
 // for, so its logit is the mean of that block's 16 fine logits and its value
 // term spreads P_c / B onto the block's 16 values: level-1 enrichment costs no
@@ -35,10 +38,11 @@ constexpr int NBUF = 3;          // groups in flight (query tiles, union lists)
 constexpr int COARSE = 32;       // pooled keys of levels >= 2 per group, at most
 constexpr int MAXPICK = 256;     // G * K_1, at most
 constexpr int MAXWORDS = 2048;   // union bitmap: level-1 blocks per slice, at most 65536
-constexpr int BATCH = 2;         // picked blocks per softmax batch (9 warps: 168 registers at most)
-constexpr int TMA_WARP = G;
-constexpr int UNION_WARP = G + 1;
-constexpr int THREADS = (G + 2) * 32;
+constexpr int CW = 2;            // consumer warps per query block: each takes every other pick
+constexpr int BATCH = 1;         // picked blocks per softmax batch
+constexpr int TMA_WARP = CW * G;
+constexpr int UNION_WARP = CW * G + 1;
+constexpr int THREADS = (CW * G + 2) * 32;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s: a wait this long means something broke
 
 struct Smem {
@@ -61,8 +65,16 @@ struct Smem {
   uint64_t qempty[NBUF];   // the group's consumers are done with the buffer
   uint64_t ufull[NBUF];    // the union list is written: union warp -> TMA warp
   uint64_t csync;          // consumer-wide barrier around the pooled-key tile
+  // a query block's second consumer warp hands its partial state to the first:
+  // O as bf16 pairs in the fragment layout ([word][lane]) and the row max and
+  // sum of rows gq, gq + 8 (log2 domain)
+  uint32_t part[G][16][32];
+  float pstat[G][4][32];
+  uint64_t mfull[G], mempty[G];
   int abort_flag;
 };
+
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of one CTA exceeds the 227 KB limit");
 
 __device__ __forceinline__ void give_up(Smem& s, int* err, int code) {
   s.abort_flag = 1;
@@ -259,10 +271,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     }
     for (int b = 0; b < NBUF; ++b) {
       ptx::mbar_init(&s.qfull[b], 2);     // the TMA bytes' arrival and the union list's arrival
-      ptx::mbar_init(&s.qempty[b], G);
+      ptx::mbar_init(&s.qempty[b], CW * G);
       ptx::mbar_init(&s.ufull[b], 1);
     }
-    ptx::mbar_init(&s.csync, G * 32);
+    for (int qb = 0; qb < G; ++qb) {
+      ptx::mbar_init(&s.mfull[qb], 1);
+      ptx::mbar_init(&s.mempty[qb], 1);
+    }
+    ptx::mbar_init(&s.csync, CW * G * 32);
     s.abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -477,7 +493,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
   }
 
   // -------------------------------------------------------------- consumers
+  // warp w takes query block w % G; half w / G of its picks (every other one)
+  // and of its pooled keys, the second half handing its state to the first
   const int gq = lane >> 2, tq4 = lane & 3;
+  const int qb = warp % G, half = warp / G;
   uint32_t cphase = 0;
   int64_t last_parent = -1;
   int it = 0;
@@ -486,7 +505,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     const uint32_t use = (uint32_t)(it / NBUF);
     const int bh = gi / groups_per_slice;
     const int a0 = (gi - bh * groups_per_slice) * G;
-    const int a = a0 + warp;
+    const int a = a0 + qb;
 
     // pooled keys of levels >= 2, once per level-2 parent (all 8 consumers)
     const int64_t parent = (int64_t)bh * g.n[1] + a0 / g.B;
@@ -508,7 +527,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
         give_up(s, err, 6);
         break;
       }
-      for (int item = threadIdx.x; item < nc * 16; item += G * 32) {
+      for (int item = threadIdx.x; item < nc * 16; item += CW * G * 32) {
         const int row = item >> 4, chunk = item & 15;
         const int l = s.crow_l[row], tok = s.crow_tok[row];
         float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
@@ -535,10 +554,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
       break;
     }
     // ring positions of this block's picks, lane j holding pick j (K_1 <= 32), ascending
-    const uint32_t my_pos = lane < K1 ? s.pickpos[b][warp * K1 + lane] : 0xffffffffu;
+    const uint32_t my_pos = lane < K1 ? s.pickpos[b][qb * K1 + lane] : 0xffffffffu;
 
     uint32_t qa[4][4];
-    const uint32_t qbase = ptx::smem_u32(s.q[b][warp]);
+    const uint32_t qbase = ptx::smem_u32(s.q[b][qb]);
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const int row = lane & 15;
@@ -555,7 +574,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
 
     // pooled keys of levels >= 2, 16 at a time
     const uint32_t ckb = ptx::smem_u32(s.ck), cvb = ptx::smem_u32(s.cv);
-    for (int k0 = 0; k0 < nc; k0 += 16) {
+    for (int k0 = 16 * half; k0 < nc; k0 += 16 * CW) {
       float sc[2][4];
       qk_16(sc, qa, ckb, k0, lane);
       float z[2][4];
@@ -598,7 +617,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     int npend = 0;
     uint32_t first_pend = 0;
     bool ok = true;
-    for (int j = 0; j < K1; ++j) {
+    for (int j = half; j < K1; j += CW) {
       const uint32_t pos = __shfl_sync(0xffffffffu, my_pos, j);
       if (pos == 0xffffffffu) continue;           // a pick outside its level: absent key
       // a held slot returns to the ring before a later pick needs the same slot
@@ -644,21 +663,58 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_mma_kernel(
     }
     if (aborted(s)) break;
 
-    // epilogue: O = acc / l, LSE = ln(sum) + max
-    const float l0 = quad_sum(st.l[0]), l1 = quad_sum(st.l[1]);
-    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-    const int64_t row0 = (int64_t)bh * g.N + (int64_t)a * 16 + gq;
-    __nv_bfloat16* o0 = o + row0 * 64;
-    __nv_bfloat16* o1 = o + (row0 + 8) * 64;
+    // epilogue: the second warp of the block hands over (m, l, O); the first
+    // merges, O = acc / l, LSE = ln(sum) + max
+    float l0 = quad_sum(st.l[0]), l1 = quad_sum(st.l[1]);
+    const uint32_t mph = (uint32_t)(it & 1);
+    if (half == 1) {
+      if (!ptx::mbar_wait_bounded(&s.mempty[qb], mph ^ 1, kWaitLimitNs)) {
+        give_up(s, err, 7);
+        break;
+      }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = j * 8 + 2 * tq4;
-      *reinterpret_cast<uint32_t*>(o0 + c) = ptx::pack_bf16(st.acc[j][0] * inv0, st.acc[j][1] * inv0);
-      *reinterpret_cast<uint32_t*>(o1 + c) = ptx::pack_bf16(st.acc[j][2] * inv1, st.acc[j][3] * inv1);
-    }
-    if (tq4 == 0) {
-      lse[row0] = (st.m[0] + log2f(l0)) * 0.6931471805599453f;
-      lse[row0 + 8] = (st.m[1] + log2f(l1)) * 0.6931471805599453f;
+      for (int jj = 0; jj < 8; ++jj) {
+        s.part[qb][2 * jj][lane] = ptx::pack_bf16(st.acc[jj][0], st.acc[jj][1]);
+        s.part[qb][2 * jj + 1][lane] = ptx::pack_bf16(st.acc[jj][2], st.acc[jj][3]);
+      }
+      s.pstat[qb][0][lane] = st.m[0];
+      s.pstat[qb][1][lane] = st.m[1];
+      s.pstat[qb][2][lane] = l0;
+      s.pstat[qb][3][lane] = l1;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.mfull[qb]);
+    } else {
+      if (!ptx::mbar_wait_bounded(&s.mfull[qb], mph, kWaitLimitNs)) {
+        give_up(s, err, 7);
+        break;
+      }
+      const float m0b = s.pstat[qb][0][lane], m1b = s.pstat[qb][1][lane];
+      const float mn0 = fmaxf(st.m[0], m0b), mn1 = fmaxf(st.m[1], m1b);
+      const float a0 = ptx::ex2(st.m[0] - mn0), a1 = ptx::ex2(st.m[1] - mn1);
+      const float b0 = ptx::ex2(m0b - mn0), b1 = ptx::ex2(m1b - mn1);
+      l0 = l0 * a0 + s.pstat[qb][2][lane] * b0;
+      l1 = l1 * a1 + s.pstat[qb][3][lane] * b1;
+      const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+      const int64_t row0 = (int64_t)bh * g.N + (int64_t)a * 16 + gq;
+      __nv_bfloat16* o0 = o + row0 * 64;
+      __nv_bfloat16* o1 = o + (row0 + 8) * 64;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const uint32_t w0 = s.part[qb][2 * jj][lane], w1 = s.part[qb][2 * jj + 1][lane];
+        const float2 p0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w0));
+        const float2 p1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w1));
+        const int c = jj * 8 + 2 * tq4;
+        *reinterpret_cast<uint32_t*>(o0 + c) =
+            ptx::pack_bf16((st.acc[jj][0] * a0 + p0.x * b0) * inv0, (st.acc[jj][1] * a0 + p0.y * b0) * inv0);
+        *reinterpret_cast<uint32_t*>(o1 + c) =
+            ptx::pack_bf16((st.acc[jj][2] * a1 + p1.x * b1) * inv1, (st.acc[jj][3] * a1 + p1.y * b1) * inv1);
+      }
+      if (tq4 == 0) {
+        lse[row0] = (mn0 + log2f(l0)) * 0.6931471805599453f;
+        lse[row0 + 8] = (mn1 + log2f(l1)) * 0.6931471805599453f;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.mempty[qb]);
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&s.qempty[b]);
