@@ -242,8 +242,9 @@ __device__ __forceinline__ void key_group_union(const Geo& g, const int32_t* __r
 
 constexpr int PREP_THREADS = 256;
 
-// Pre-pass, one CTA per level-2 token t (query groups 2t, 2t + 1; key groups
-// 2t, 2t + 1 are the same 16 blocks as keys):
+// Pre-pass, two CTAs per level-2 token t (query groups 2t, 2t + 1; key groups
+// 2t, 2t + 1 are the same 16 blocks as keys), the first doing the lists and
+// the tile, the second D:
 //   * warps 0, 1: the unions of the two query groups' pick lists;
 //   * warps 2, 3: the unions of the two key groups' CSC lists (for the
 //     key-major pass);
@@ -265,10 +266,12 @@ __global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32
                                                               float* __restrict__ Dws, unsigned char* __restrict__ ctile,
                                                               int nc) {
   __shared__ int stage[4][UNION_STAGE];
-  const int t = blockIdx.x;
+  // Two blocks per token, interleaved: the odd one streams D (bound by DRAM),
+  // the even one merges the unions and builds the pooled-key tile (bound by
+  // latency), so that neither holds the other's resources.
+  const int t = blockIdx.x >> 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane, stage[warp]);
-  else if (warp < 4) key_group_union(g, offs, qlist, ulist_kv, ucount_kv, 2 * t + warp - 2, lane, stage[warp]);
+  if (blockIdx.x & 1) {
   const int64_t row0 = (int64_t)t * 2 * QG * 16;
 #pragma unroll 2
   for (int it = 0; it < 8; ++it) {
@@ -289,6 +292,10 @@ __global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
     if ((lane & 7) == 0) Dws[gr] = acc;
   }
+  return;
+  }
+  if (warp < 2) group_union(g, idx, ulist, ucount, 2 * t + warp, lane, stage[warp]);
+  else if (warp < 4) key_group_union(g, offs, qlist, ulist_kv, ucount_kv, 2 * t + warp - 2, lane, stage[warp]);
   if (nc <= 0) return;
   const int n1 = g.n[1];
   const int bh = (2 * t * QG) / n1;
@@ -979,7 +986,7 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   const int ngroups = (int)((int64_t)g.BH * g.n[1] / bwdq::QG);
   const int ntokens = ngroups / 2;
   if (ntokens == 0) return cudaSuccess;
-  bwdq::q_prep_kernel<<<ntokens, bwdq::PREP_THREADS, 0, s>>>(g, idx, (const __nv_bfloat16*)o,
+  bwdq::q_prep_kernel<<<2 * ntokens, bwdq::PREP_THREADS, 0, s>>>(g, idx, (const __nv_bfloat16*)o,
                                                              (const __nv_bfloat16*)dO, pyrK, pyrV, offs, qlist,
                                                              ws.ulist, ws.ucount, ws.ulist_kv, ws.ucount_kv, ws.D,
                                                              ws.ctile, nc);
