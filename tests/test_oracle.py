@@ -120,7 +120,8 @@ def _brute_select(p, pq, pk):
     return out
 
 
-@pytest.mark.parametrize("H,W,B,L,K", [(32, 32, 16, 2, 4), (64, 64, 16, 3, 3), (16, 16, 4, 3, 2), (32, 32, 4, 3, 5)])
+@pytest.mark.parametrize("H,W,B,L,K", [(32, 32, 16, 2, 4), (64, 64, 16, 3, 3), (16, 16, 4, 3, 2), (32, 32, 4, 3, 5),
+                                      (32, 32, 16, 1, 5)])
 def test_select_equals_brute_force(H, W, B, L, K):
     rng = np.random.default_rng(H + L + K)
     p = oracle.Problem(H=H, W=W, d=6, B=B, L=L, K=K)
@@ -326,3 +327,82 @@ def test_gradient_sums_hold():
     _, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g)
     np.testing.assert_allclose(dv.sum(axis=1), g.sum(axis=1), rtol=1e-12, atol=1e-11)
     np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-11)
+
+
+# ------------------------------------------- one level, enrichment variants
+
+def test_single_level_is_block_top_k_attention():
+    # With L = 1 the method is the single-level block top-K attention that the
+    # Trainable LLSA summary (§一) compares against: every query block scores
+    # all n_1 key blocks by the dot product of the two block means and attends,
+    # at full resolution, to the tokens of its K best blocks.  Written out here
+    # with explicit means, a full score matrix and a stable sort.
+    rng = np.random.default_rng(13)
+    p = oracle.Problem(H=32, W=32, d=8, B=16, L=1, K=3, enrich_mask=0)
+    q, k, v = (_rand(rng, 1, p.N, p.d) for _ in range(3))
+    r = oracle.forward(p, q, k, v)
+    nb = p.N // 16
+    qm, km = q[0].reshape(nb, 16, p.d).mean(1), k[0].reshape(nb, 16, p.d).mean(1)
+    S = qm @ km.T
+    for a in range(nb):
+        order = sorted(range(nb), key=lambda j: (-S[a, j], j))
+        blocks = sorted(order[:3])
+        assert r["idx"][0][0, a].tolist() == blocks
+        keys = [c * 16 + t for c in blocks for t in range(16)]
+        for i in range(a * 16, a * 16 + 16, 5):
+            o, lse = _dense(q[:, i:i + 1], k[:, keys], v[:, keys], p.scale)
+            np.testing.assert_allclose(r["o"][0, i], o[0, 0], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(r["lse"][0, i], lse[0, 0], rtol=1e-12)
+
+
+@pytest.mark.parametrize("mask", [0b00, 0b01, 0b10, 0b11])
+def test_enrichment_levels_add_their_pooled_tokens(mask):
+    # Each enriched level l adds, for query i, the K_l pooled tokens picked by
+    # i's level-l ancestor with logit bias ln B^l (weight B^l, Trainable LLSA
+    # summary §四); the fine keys of the level-1 picks are always attended.
+    # Written out per query with explicit means of the B^l member tokens.
+    rng = np.random.default_rng(14 + mask)
+    p = oracle.Problem(H=32, W=32, d=8, B=16, L=2, K=2, enrich_mask=mask)
+    q, k, v = (_rand(rng, 1, p.N, p.d) for _ in range(3))
+    r = oracle.forward(p, q, k, v)
+    idx = r["idx"]
+    for i in range(0, p.N, 29):
+        keys = [c * 16 + t for c in idx[0][0, i // 16] for t in range(16)]
+        zk, zv = [k[0, j] for j in keys], [v[0, j] for j in keys]
+        bias = [0.0] * len(keys)
+        for l in (1, 2):
+            if not (mask >> (l - 1)) & 1:
+                continue
+            for c in idx[l - 1][0, i // 16 ** l]:
+                members = slice(c * 16 ** l, (c + 1) * 16 ** l)
+                zk.append(k[0, members].mean(0))
+                zv.append(v[0, members].mean(0))
+                bias.append(l * np.log(16.0))
+        z = np.array(zk) @ q[0, i] * p.scale + np.array(bias)
+        lse = np.log(np.exp(z - z.max()).sum()) + z.max()
+        o = np.exp(z - lse) @ np.array(zv)
+        np.testing.assert_allclose(r["o"][0, i], o, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(r["lse"][0, i], lse, rtol=1e-12)
+
+
+def test_single_level_backward_matches_finite_differences():
+    # L = 1 with its one level enriched; index lists frozen; fp64 central
+    # differences on a sample of coordinates.
+    rng = np.random.default_rng(15)
+    p = oracle.Problem(H=16, W=16, d=8, B=16, L=1, K=3)
+    q, k, v, g = (_rand(rng, 1, p.N, p.d) for _ in range(4))
+    r = oracle.forward(p, q, k, v)
+    idx = r["idx"]
+    dq, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], idx, g)
+    h = 1e-6
+    for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for e in rng.choice(p.N * p.d, size=120, replace=False):
+            t, c = divmod(int(e), p.d)
+            args = {"q": q, "k": k, "v": v}
+            plus = {n_: a.copy() for n_, a in args.items()}
+            minus = {n_: a.copy() for n_, a in args.items()}
+            plus[which][0, t, c] += h
+            minus[which][0, t, c] -= h
+            fd = (_loss(p, plus["q"], plus["k"], plus["v"], idx, g)
+                  - _loss(p, minus["q"], minus["k"], minus["v"], idx, g)) / (2 * h)
+            assert abs(fd - grad[0, t, c]) <= 1e-6 * max(1.0, abs(fd)), (which, t, c, fd, grad[0, t, c])
