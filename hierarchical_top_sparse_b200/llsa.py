@@ -35,7 +35,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "alignment", 4: "worksp
 
 EXPORTS = ("llsa_status_string", "llsa_validate", "llsa_level_sizes", "llsa_query_sizes", "llsa_reorder",
            "llsa_pool", "llsa_select", "llsa_select_level", "llsa_attn_fwd", "llsa_index_transpose",
-           "llsa_attn_bwd", "llsa_device_error", "llsa_kernel_launches", "llsa_index_transpose_noalloc")
+           "llsa_attn_bwd", "llsa_device_error", "llsa_kernel_launches", "llsa_index_transpose_noalloc",
+           "llsa_selftest_wait_timeout")
 
 
 class LLSAError(RuntimeError):
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "llsa_attn_bwd": ([P] + [vp] * 16, i32),
             "llsa_device_error": ([vp, ctypes.POINTER(i32)], i32),
             "llsa_kernel_launches": ([], ctypes.c_uint64),
+            "llsa_selftest_wait_timeout": ([ctypes.c_uint, i32, i32, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -227,6 +229,12 @@ def device_error(stream=None) -> int:
     if st not in (0, 6):
         raise LLSAError(st, "device_error")
     return code.value
+
+
+def selftest_wait_timeout(limit_us: int, code: int, arrive: bool = False, stream=None):
+    """Launches the timeout-path self-test (llsa_selftest_wait_timeout)."""
+    _check(lib().llsa_selftest_wait_timeout(int(limit_us), int(code), int(bool(arrive)), _stream(stream)),
+           "selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------ layouts

@@ -191,6 +191,17 @@ uint64_t llsa_kernel_launches(void);
  * wait gave up; returns LLSA_ERR_TIMEOUT when one did. */
 llsa_status llsa_device_error(llsa_stream stream, int* code);
 
+/* Self-test of the timeout path of the bounded device waits: launches one
+ * thread on `stream` that waits, with the same bounded wait the pipelined
+ * kernels use, on an mbarrier phase that nothing completes (arrive = 0) or
+ * that it completed itself first (arrive = 1).  When the wait gives up after
+ * limit_us microseconds the device error word is set to `code`, so that the
+ * next llsa_device_error returns LLSA_ERR_TIMEOUT with *code = code; with
+ * arrive = 1 it stays 0.  Neither faults nor hangs the GPU.  limit_us in
+ * [1, 1000000], code != 0, arrive in {0, 1}, else LLSA_ERR_ARG before any
+ * launch. */
+llsa_status llsa_selftest_wait_timeout(unsigned limit_us, int code, int arrive, llsa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

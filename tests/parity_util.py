@@ -111,6 +111,8 @@ class GpuRun:
         if backward:
             pipe.backward_pass(dq_, dk_, dv_, dg_)
         torch.cuda.synchronize()
+        # no bounded device wait gave up during the run (reading clears the word)
+        assert llsa.device_error() == 0, "a bounded device wait gave up"
         p = self.p
         self.pyrQ = [to_np(t) for t in llsa.level_views(p, pipe.pyrQ, p.d)]
         self.pyrK = [to_np(t) for t in llsa.level_views(p, pipe.pyrK, p.d)]

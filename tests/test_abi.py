@@ -103,6 +103,12 @@ def test_entry_points_reject_null_and_misaligned_buffers_before_launch(L):
     assert L.llsa_pool(ctypes.byref(bad_p), good, good, None) == 2
 
 
+def test_timeout_selftest_rejects_bad_arguments_before_launch(L):
+    # limit_us in [1, 1e6], code != 0, arrive in {0, 1}: LLSA_ERR_ARG, no CUDA call
+    for args in ((0, 5, 0), (1000001, 5, 0), (10, 0, 0), (10, 5, 2), (10, 5, -1)):
+        assert L.llsa_selftest_wait_timeout(*args, None) == 1, args
+
+
 def test_status_strings(L):
     for s in range(8):
         assert llsa.status_string(s)
