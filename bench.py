@@ -31,9 +31,30 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-WORKLOAD = dict(name="px256", batch=2, heads=6, H=256, W=256, d=64, B=16, L=4, K=8, sigma=4.0)
-METRIC = "LLSA fwd+bwd tokens/s at 256² pixels (N=65536); % of roofline"
+# The workload the metric is quoted on (the default), and the other forward +
+# backward workloads that --workload can time instead: the 128 x 128 and
+# 512 x 512 training-step sizes, and at 256 x 256 the block-size and top-K
+# variants the pages ablate (B = 64 runs on the CUDA-core kernels).
+WORKLOADS = {
+    "px256": dict(name="px256", batch=2, heads=6, H=256, W=256, d=64, B=16, L=4, K=8, sigma=4.0),
+    "px128": dict(name="px128", batch=8, heads=6, H=128, W=128, d=64, B=16, L=3, K=8, sigma=4.0),
+    "px512": dict(name="px512", batch=1, heads=16, H=512, W=512, d=64, B=16, L=4, K=8, sigma=8.0),
+    "px256_K16": dict(name="px256_K16", batch=2, heads=6, H=256, W=256, d=64, B=16, L=4, K=16, sigma=4.0),
+    "px256_B64": dict(name="px256_B64", batch=2, heads=6, H=256, W=256, d=64, B=64, L=2, K=8, sigma=4.0),
+}
+WORKLOAD = WORKLOADS["px256"]
+METRIC_PX256 = "LLSA fwd+bwd tokens/s at 256² pixels (N=65536); % of roofline"
+METRIC = METRIC_PX256
 UNIT = "tokens/s"
+
+
+def select_workload(name: str):
+    """Makes `name` the timed workload (module state read by every arm)."""
+    global WORKLOAD, METRIC
+    WORKLOAD = w = WORKLOADS[name]
+    METRIC = METRIC_PX256 if name == "px256" else (
+        f"LLSA fwd+bwd tokens/s at {w['H']}x{w['W']} pixels (N={w['H'] * w['W']}, B={w['B']}, K={w['K']}); "
+        "% of roofline")
 
 
 def config_desc(extra=None):
@@ -43,7 +64,8 @@ def config_desc(extra=None):
                      f"pool+select+attn_fwd+index_transpose+attn_bwd per step",
          "tokens_per_step_per_gpu": w["batch"] * w["H"] * w["W"],
          "inputs": f"seeded smooth fields (Gaussian sigma={w['sigma']} px, +0.1 white noise), dO ~ N(0,1)",
-         "l2": "no flush: inputs larger than L2 (Q, K, V, dO = 403 MB per step vs 126 MB L2)"}
+         "l2": f"no flush: inputs larger than L2 (Q, K, V, dO = "
+               f"{4 * w['batch'] * w['heads'] * w['H'] * w['W'] * w['d'] * 2 / 1e6:.0f} MB per step vs 126 MB L2)"}
     if extra:
         c.update(extra)
     return c
@@ -214,7 +236,7 @@ def traffic_record(kernel_stage: str):
     """DRAM bytes per launch from the committed ncu summary, if the stage's
     kernel sources are unchanged since the capture; else None."""
     path = os.path.join(ROOT, "profiles", "traffic_px256.txt")
-    if not os.path.exists(path):
+    if WORKLOAD["name"] != "px256" or not os.path.exists(path):   # the record covers the 256 x 256 workload
         return None
     digest = sources_digest(kernel_stage)
     for line in open(path):
@@ -532,7 +554,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="px256",
+                    help="the workload to time (default: the one the metric is quoted on)")
     args = ap.parse_args()
+    select_workload(args.workload)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     rank, local, world, pg = dist_setup(args.gpus)
