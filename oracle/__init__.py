@@ -18,9 +18,12 @@ Arrays use the same shapes as the CUDA path's public API, but per level:
 Pinning status of every routine (the tests in ``tests/test_oracle.py``):
   reorder_index / reorder   pinned: bijection, square-tile property, hand-worked table
   pool                      pinned: direct block means, raster-square means
-  select                    pinned: brute-force top-K, child invariant, ties, K = all
-  attn_fwd                  pinned: dense softmax attention at K = all; B^l copies identity
-  attn_bwd                  pinned: central finite differences; dense autograd at K = all
+  select                    pinned: brute-force top-K, child invariant, ties, K = all; one level =
+                            block top-K by the block means
+  attn_fwd                  pinned: dense softmax attention at K = all; B^l copies identity; each
+                            enrichment mask against explicitly listed pooled tokens; one level
+  attn_bwd                  pinned: central finite differences (also at one level); dense autograd
+                            at K = all
   attn_dq_rows              pinned: equals the rows of attn_bwd's dQ
   index_transpose           pinned: exact inverse of the query-major lists
 """
