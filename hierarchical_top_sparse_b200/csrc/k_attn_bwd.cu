@@ -24,11 +24,16 @@
 namespace llsa {
 
 constexpr int kBwdCoarseMax = 32;   // pooled keys of levels >= 2 per query block that the passes hold
+// Largest level-1 list the tensor-core passes take: the K = all lists of a
+// 256 x 256 image (every one of its 4096 blocks), the largest case the GPU
+// tests run them on.  Longer lists go to the CUDA-core kernels.
+constexpr int kBwdMaxK1 = 4096;
 
 bool attn_bwd_mma_supported(const Geo& g) {
   if (!g.bf16 || g.d != 64 || g.B != 16) return false;
   if (g.n[1] % 16) return false;    // whole level-2 tokens: two groups of 8 query blocks
-  if (g.Kl[1] < 1) return false;
+  if (g.n[1] >= (1 << 23)) return false;   // union entries pack (block << 8) | mask into 32 bits
+  if (g.Kl[1] < 1 || g.Kl[1] > kBwdMaxK1) return false;
   int nc = 0;
   for (int l = 2; l <= g.L; ++l)
     if ((g.emask >> (l - 1)) & 1u) nc += g.Kl[l];

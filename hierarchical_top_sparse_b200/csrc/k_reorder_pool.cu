@@ -44,6 +44,29 @@ __global__ void reorder_kernel(const uint4* __restrict__ in, uint4* __restrict__
   }
 }
 
+// The same with 32-bit index arithmetic, for tile sides t = 2^lt and fewer
+// than 2^32 vectors in all: per vector three 32-bit divisions and shifts, so
+// that the copy stays bound by memory rather than by the index math.
+__global__ void reorder32_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, uint32_t N, uint32_t vec,
+                                 uint32_t total, int lt, int L, uint32_t W, uint32_t Gw, int to_hier) {
+  const uint32_t tmask = (1u << lt) - 1u;
+  const int ltL = lt * L;
+  for (uint32_t e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const uint32_t row = e / vec, vcol = e - row * vec;
+    const uint32_t bh = row / N, r = row - bh * N;         // raster position within the slice
+    const uint32_t y = r / W, x = r - y * W;
+    uint32_t h = ((y >> ltL) * Gw + (x >> ltL)) << (2 * ltL);
+    for (int l = 0; l < L; ++l)
+      h |= ((((y >> (lt * l)) & tmask) << lt) | ((x >> (lt * l)) & tmask)) << (2 * lt * l);
+    const size_t base = (size_t)bh * N;
+    const size_t rr = (base + r) * vec + vcol, hh = (base + h) * vec + vcol;
+    if (to_hier)
+      out[hh] = in[rr];
+    else
+      out[rr] = in[hh];
+  }
+}
+
 static int grid_for(int64_t work, int threads) {
   int64_t blocks = (work + threads - 1) / threads;
   int64_t cap = 148ll * 16;
@@ -53,6 +76,17 @@ static int grid_for(int64_t work, int threads) {
 cudaError_t launch_reorder(const Geo& g, const void* in, void* out, int to_hier, cudaStream_t s) {
   int vec = g.d * (g.bf16 ? 2 : 4) / 16;
   int64_t total = (int64_t)g.BH * g.N * vec;
+  int lt = 0;
+  while ((1 << lt) < g.t) ++lt;
+  if ((1 << lt) == g.t && total < (1ll << 32)) {
+    int64_t tl = 1;
+    for (int l = 0; l < g.L; ++l) tl *= g.t;
+    reorder32_kernel<<<grid_for(total, 256), 256, 0, s>>>((const uint4*)in, (uint4*)out, (uint32_t)g.N,
+                                                          (uint32_t)vec, (uint32_t)total, lt, g.L, (uint32_t)g.W,
+                                                          (uint32_t)(g.W / tl), to_hier);
+    note_launches(1);
+    return cudaGetLastError();
+  }
   reorder_kernel<<<grid_for(total, 256), 256, 0, s>>>((const uint4*)in, (uint4*)out, g.N, vec, total, g.t,
                                                       g.L, g.W, g.Bl[g.L], to_hier);
   note_launches(1);

@@ -9,8 +9,6 @@
 // The scatter order is arbitrary, so a last pass writes each key's ids in
 // ascending order (short ranges by an in-register rank, long ranges through a
 // shared-memory bitmap of the query ids).
-#include <mutex>
-
 #include "llsa_internal.cuh"
 
 namespace llsa {
@@ -227,32 +225,21 @@ cudaError_t launch_index_transpose(const Geo& g, const int32_t* idx, int32_t* of
 // fixed device array owned by this library instead of a caller buffer.  The
 // array is a file-scope __device__ object, so every GPU that loads the library
 // holds kNoAllocScratchBytes of it until the process exits.  Host code cannot
-// use the symbol's name as a device address: its address is looked up once
-// per device with cudaGetSymbolAddress (on the first call made while that
-// device is current) and cached.
+// use the symbol's name as a device address: every call looks up its address
+// on the current device with cudaGetSymbolAddress (a host-side lookup, no
+// launch), so that a device reset between calls cannot leave a stale address.
 
 namespace llsa {
 
 constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
-constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[kNoAllocMaxDevices];
-
 // Device address of g_noalloc_scratch on the current device.
 static llsa_status noalloc_scratch(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LLSA_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return LLSA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LLSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LLSA_ERR_CUDA;
+  *out = ptr;
   return LLSA_OK;
 }
 

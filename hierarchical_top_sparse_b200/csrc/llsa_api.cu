@@ -265,6 +265,13 @@ llsa_status llsa_attn_bwd(const llsa_problem* p, const void* q, const void* k, c
                                         workspace, (cudaStream_t)stream));
 }
 
+llsa_status llsa_attn_paths(const llsa_problem* p, int* fwd_tc, int* bwd_tc) {
+  LLSA_GEO(p, g);
+  if (fwd_tc) *fwd_tc = llsa::attn_fwd_mma_supported(g) ? 1 : 0;
+  if (bwd_tc) *bwd_tc = llsa::attn_bwd_mma_supported(g) ? 1 : 0;
+  return LLSA_OK;
+}
+
 uint64_t llsa_kernel_launches(void) { return (uint64_t)llsa::g_launches.load(std::memory_order_relaxed); }
 
 llsa_status llsa_device_error(llsa_stream stream, int* code) {

@@ -36,7 +36,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "alignment", 4: "worksp
 EXPORTS = ("llsa_status_string", "llsa_validate", "llsa_level_sizes", "llsa_query_sizes", "llsa_reorder",
            "llsa_pool", "llsa_select", "llsa_select_level", "llsa_attn_fwd", "llsa_index_transpose",
            "llsa_attn_bwd", "llsa_device_error", "llsa_kernel_launches", "llsa_index_transpose_noalloc",
-           "llsa_selftest_wait_timeout")
+           "llsa_selftest_wait_timeout", "llsa_attn_paths")
 
 
 class LLSAError(RuntimeError):
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "llsa_device_error": ([vp, ctypes.POINTER(i32)], i32),
             "llsa_kernel_launches": ([], ctypes.c_uint64),
             "llsa_selftest_wait_timeout": ([ctypes.c_uint, i32, i32, vp], i32),
+            "llsa_attn_paths": ([P, ctypes.POINTER(i32), ctypes.POINTER(i32)], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -216,6 +217,14 @@ def attn_bwd(p: Problem, q, k, v, o, dO, lse, pyrK, pyrV, idx, offs, qlist, dq, 
     _check(lib().llsa_attn_bwd(ctypes.byref(p.c()), *[_ptr(t) for t in (q, k, v, o, dO, lse, pyrK, pyrV, idx, offs,
                                                                           qlist, dq, dk, dv, workspace)],
                                _stream(stream)), "attn_bwd")
+
+
+def attn_paths(p: Problem) -> dict:
+    """Which kernels attn_fwd / attn_bwd run for p: "tensor" or "cuda-core"."""
+    f, b = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().llsa_attn_paths(ctypes.byref(p.c()), ctypes.byref(f), ctypes.byref(b)), "attn_paths")
+    name = {1: "tensor", 0: "cuda-core"}
+    return {"fwd": name[f.value], "bwd": name[b.value]}
 
 
 def kernel_launches() -> int:

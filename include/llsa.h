@@ -31,6 +31,18 @@
  * * Host-detectable errors (bad shapes, NULL or misaligned pointers,
  *   unsupported sizes) return a status before anything is launched.  A
  *   launch failure returns LLSA_ERR_CUDA.  No exception crosses the ABI.
+ * * Buffer sizes are queried with llsa_query_sizes (one call returns every
+ *   size, the workspaces included); device-side timeouts are read with
+ *   llsa_device_error.  The main entry points take no size arguments: their
+ *   buffers must have the queried sizes.  LLSA_ERR_WORKSPACE is returned only
+ *   by llsa_index_transpose_noalloc, whose scratch has a fixed size.
+ * * Pooled tokens: pyrK / pyrV passed to the attention calls must be what
+ *   llsa_pool wrote for the same k / v.  Level 1 is then the exact mean of
+ *   the B key (value) rows it stands for, and the tensor-core kernels (bf16,
+ *   d = 64, B = 16) use that identity: they form level-1 pooled logits and
+ *   values from k / v themselves and do not read level 1 of pyrK / pyrV.  The
+ *   CUDA-core kernels (every other problem) read it.  Levels >= 2 are read by
+ *   both.
  */
 #ifndef LLSA_H
 #define LLSA_H
@@ -50,7 +62,7 @@ typedef enum {
   LLSA_ERR_ARG = 1,          /* NULL pointer or invalid field */
   LLSA_ERR_SHAPE = 2,        /* image does not tile into sqrt(B)^L squares, or sizes overflow */
   LLSA_ERR_ALIGN = 3,        /* a buffer is not 16-byte aligned */
-  LLSA_ERR_WORKSPACE = 4,    /* reserved: workspace too small */
+  LLSA_ERR_WORKSPACE = 4,    /* the fixed scratch of llsa_index_transpose_noalloc is too small */
   LLSA_ERR_CUDA = 5,         /* a CUDA launch or runtime call failed */
   LLSA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up (see llsa_device_error) */
   LLSA_ERR_UNSUPPORTED = 7   /* valid problem outside what the kernels implement */
@@ -159,9 +171,11 @@ llsa_status llsa_index_transpose(const llsa_problem* p, const int32_t* idx, int3
  * that (transpose_scratch_bytes > 16 MiB) is rejected with
  * LLSA_ERR_WORKSPACE before anything is launched.  Nothing is allocated:
  * no cudaMalloc, no cudaFree.
- * The first call on a device, made while that device is current, looks up
- * the array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture.  All calls share the one array and it
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, a host-side lookup that launches nothing), so a
+ * device reset between calls leaves no stale address behind.  The first call
+ * on a device may load this library's device code there; make it before any
+ * stream capture.  All calls share the one array and it
  * keeps whatever the last call left there (the parts that must start at zero
  * are cleared by every call), so two calls whose work overlaps on the GPU --
  * on different streams, or from different threads -- race and must be
@@ -182,13 +196,21 @@ llsa_status llsa_attn_bwd(const llsa_problem* p, const void* q, const void* k, c
                           const float* pyrV, const int32_t* idx, const int32_t* offs, const int32_t* qlist,
                           void* dq, void* dk, void* dv, void* workspace, llsa_stream stream);
 
+/* Which kernels llsa_attn_fwd and llsa_attn_bwd run for *p (host only, no
+ * launch): *fwd_tc / *bwd_tc = 1 for the tensor-core kernels (tcgen05 /
+ * TMEM, bf16, d = 64, B = 16, within the sizes they support), 0 for the
+ * CUDA-core kernels.  Either pointer may be NULL. */
+llsa_status llsa_attn_paths(const llsa_problem* p, int* fwd_tc, int* bwd_tc);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (all entry points, all streams); for accounting in benchmarks. */
 uint64_t llsa_kernel_launches(void);
 
 /* Waits for `stream`, then reads and clears the device-side error word that
  * bounded waits inside the kernels set when they give up.  *code = 0 when no
- * wait gave up; returns LLSA_ERR_TIMEOUT when one did. */
+ * wait gave up; returns LLSA_ERR_TIMEOUT when one did.  There is one word
+ * per device, shared by every stream and thread of the process: a code
+ * cannot be attributed to one stream, and a read clears it for all. */
 llsa_status llsa_device_error(llsa_stream stream, int* code);
 
 /* Self-test of the timeout path of the bounded device waits: launches one

@@ -26,6 +26,8 @@ Pinning status of every routine (the tests in ``tests/test_oracle.py``):
                             at K = all
   attn_dq_rows              pinned: equals the rows of attn_bwd's dQ
   index_transpose           pinned: exact inverse of the query-major lists
+  dense_attention           pinned: torch autograd (fp64) on CPU; equals attn_fwd / attn_bwd at K = all
+                            without enrichment
 """
 from __future__ import annotations
 
@@ -329,6 +331,72 @@ def index_transpose(p: Problem, idx: Sequence[np.ndarray]):
         a += n[l] + 1
         b += n[l] * kl[l]
     return lo, lq
+
+
+def dense_attention(q, k, v, scale: float, dO=None, rows=None, keys=None, chunk: int = 1024):
+    """Plain softmax attention of every query over every key of its slice, the
+    closed form that LLSA reduces to when every block is selected at every
+    level and no pooled token joins ("Trainable Log-linear Sparse Attention"
+    summary, §一: the method restricts dense attention to the selected
+    blocks).  fp64, with library matrix products and exponentials (torch CPU
+    ops) over chunks of query rows; nothing else is reordered.
+
+      z_ij = scale * q_i . k_j,  lse_i = log sum_j exp z_ij,  P_ij = exp(z_ij - lse_i)
+      o_i = sum_j P_ij v_j
+      dP_ij = dO_i . v_j,  D_i = dO_i . o_i,  dz_ij = P_ij (dP_ij - D_i)
+      dq_i = scale * sum_j dz_ij k_j,  dk_j = scale * sum_i dz_ij q_i,  dv_j = sum_i P_ij dO_i
+
+    q, k, v, dO: [BH, N, d].  ``rows`` (query positions, default all) selects
+    the rows of o, lse and dq that are returned ([BH, len(rows), ...]);
+    ``keys`` (key positions) asks for dk and dv of those keys, which need every
+    query row of the slice.  Returns a dict with o, lse and, when dO is given,
+    dq (and dk, dv when keys are given)."""
+    import torch
+    qs, ks, vs = (torch.from_numpy(_as_slices(a, 2)) for a in (q, k, v))
+    gs = None if dO is None else torch.from_numpy(_as_slices(dO, 2))
+    BH, N, d = qs.shape
+    rows_t = torch.arange(N) if rows is None else torch.from_numpy(np.asarray(rows, dtype=np.int64))
+    keys_t = None if keys is None else torch.from_numpy(np.asarray(keys, dtype=np.int64))
+    out = {"o": np.empty((BH, len(rows_t), d)), "lse": np.empty((BH, len(rows_t)))}
+    if gs is not None:
+        out["dq"] = np.empty((BH, len(rows_t), d))
+        if keys_t is not None:
+            out["dk"] = np.zeros((BH, len(keys_t), d))
+            out["dv"] = np.zeros((BH, len(keys_t), d))
+
+    def block(s, r):
+        z = (qs[s, r] @ ks[s].T) * scale
+        lse = torch.logsumexp(z, dim=1)
+        P = torch.exp(z - lse[:, None])
+        o = P @ vs[s]
+        return z, lse, P, o
+
+    for s in range(BH):
+        for c0 in range(0, len(rows_t), chunk):
+            r = rows_t[c0:c0 + chunk]
+            _, lse, P, o = block(s, r)
+            out["o"][s, c0:c0 + len(r)] = o.numpy()
+            out["lse"][s, c0:c0 + len(r)] = lse.numpy()
+            if gs is not None:
+                dP = gs[s, r] @ vs[s].T
+                D = (gs[s, r] * o).sum(dim=1)
+                dz = P * (dP - D[:, None])
+                out["dq"][s, c0:c0 + len(r)] = (scale * (dz @ ks[s])).numpy()
+        if gs is not None and keys_t is not None:
+            dk = torch.zeros((len(keys_t), d), dtype=torch.float64)
+            dv = torch.zeros((len(keys_t), d), dtype=torch.float64)
+            for c0 in range(0, N, chunk):
+                r = torch.arange(c0, min(N, c0 + chunk))
+                _, lse, P, o = block(s, r)
+                PJ = P[:, keys_t]
+                dPJ = gs[s, r] @ vs[s, keys_t].T
+                D = (gs[s, r] * o).sum(dim=1)
+                dzJ = PJ * (dPJ - D[:, None])
+                dk += scale * (dzJ.T @ qs[s, r])
+                dv += PJ.T @ gs[s, r]
+            out["dk"][s] = dk.numpy()
+            out["dv"][s] = dv.numpy()
+    return out
 
 
 def forward(p: Problem, q_hier, k_hier, v_hier):

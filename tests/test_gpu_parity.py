@@ -76,19 +76,58 @@ def check_attention(run: GpuRun, backward: bool, sel=slice(None)):
     return res
 
 
-def check_end_to_end(run: GpuRun, sel=slice(None), min_match=0.99):
-    """The oracle's own selection; rows whose lists all agree must agree in O."""
-    op, dt = run.op, run.case.dtype
-    r = oracle.forward(op, run.qh[sel], run.kh[sel], run.vh[sel])
+def agreeing_rows(op, gpu_idx, ora_idx):
+    """[BH, N] bool: fine rows whose lists (every level's list of every one of
+    their ancestors) are identical in the two selections."""
     n, _ = op.levels()
-    BH = r["o"].shape[0]
-    same = np.ones((BH, n[0]), bool)
+    same = np.ones((gpu_idx[0].shape[0], n[0]), bool)
     for l in range(1, op.L + 1):
-        eq = np.all(r["idx"][l - 1] == run.idx[l - 1][sel], axis=-1)          # [BH, n_l]
+        eq = np.all(gpu_idx[l - 1] == ora_idx[l - 1], axis=-1)          # [BH, n_l]
         same &= np.repeat(eq, op.B ** l, axis=1)
+    return same
+
+
+def agreeing_keys(op, gpu_idx, ora_idx, same):
+    """[BH, N] bool: fine keys whose gradient is formed by the same query rows,
+    all of them agreeing rows, in both selections: no query token with a
+    disagreeing row picked the key's block (level 1), nor, for every enriched
+    level l >= 2, the key's level-l ancestor, in either selection."""
+    n, _ = op.levels()
+    BH, N = same.shape
+    ok = np.ones((BH, N), bool)
+    for l in range(1, op.L + 1):
+        if l > 1 and not (op.enrich_mask >> (l - 1)) & 1:
+            continue
+        rowok = same.reshape(BH, n[l], op.B ** l).all(axis=2)          # [BH, n_l] query tokens
+        bad = np.zeros((BH, n[l]), bool)
+        for s, a in zip(*np.nonzero(~rowok)):
+            for lists in (gpu_idx, ora_idx):
+                u = lists[l - 1][s, a]
+                bad[s, u[(u >= 0) & (u < n[l])]] = True
+        ok &= ~np.repeat(bad, op.B ** l, axis=1)
+    return ok
+
+
+def check_end_to_end(run: GpuRun, sel=slice(None), min_match=0.99, grads=True):
+    """The oracle's own selection, forward and backward: rows whose lists all
+    agree must agree in O and dQ; keys whose gradients are formed by agreeing
+    rows only must agree in dK and dV."""
+    op, dt = run.op, run.case.dtype
+    qh, kh, vh = run.qh[sel], run.kh[sel], run.vh[sel]
+    r = oracle.forward(op, qh, kh, vh)
+    gpu_idx = [a[sel] for a in run.idx]
+    same = agreeing_rows(op, gpu_idx, r["idx"])
     frac = same.mean()
     assert frac >= min_match, f"only {frac:.4f} of the rows have identical index lists"
     assert_close("O (end to end)", run.o[sel][same], r["o"][same], dt)
+    assert_close("LSE (end to end)", run.lse[sel][same], r["lse"][same], dt)
+    if grads:
+        dq, dk, dv, _, _ = oracle.attn_bwd(op, qh, kh, vh, r["pyrK"], r["pyrV"], r["idx"], run.gh[sel])
+        kok = agreeing_keys(op, gpu_idx, r["idx"], same)
+        assert kok.mean() >= min_match - 0.05, f"only {kok.mean():.4f} of the keys are formed by agreeing rows"
+        assert_close("dQ (end to end)", run.dq[sel][same], dq[same], dt)
+        assert_close("dK (end to end)", run.dk[sel][kok], dk[kok], dt)
+        assert_close("dV (end to end)", run.dv[sel][kok], dv[kok], dt)
     return frac
 
 
@@ -153,6 +192,69 @@ def test_dense_when_k_covers_everything():
     check_transpose(run)
 
 
+def check_selects_everything(run: GpuRun):
+    """K at least every candidate count: every list holds every token of its level."""
+    n, kl = run.op.levels()
+    for l in range(1, run.op.L + 1):
+        assert kl[l] == n[l]
+        got = run.idx[l - 1]
+        np.testing.assert_array_equal(got, np.broadcast_to(np.arange(n[l], dtype=np.int32), got.shape))
+
+
+# bf16 K = all without enrichment, through the tensor-core kernels: every
+# level-1 list holds every block, so the backward's unions span the whole
+# slice (256 and 1024 blocks); compared with dense softmax attention
+DENSE_BF16 = {
+    "px64_dense": Case(batch=1, heads=2, H=64, W=64, L=3, K=10 ** 6, enrich_mask=0),
+    "px128_dense": Case(batch=1, heads=2, H=128, W=128, L=3, K=10 ** 6, enrich_mask=0),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DENSE_BF16))
+def test_dense_bf16_on_the_tensor_cores(name):
+    from hierarchical_top_sparse_b200 import llsa
+    case = DENSE_BF16[name]
+    p, _ = case.problems()
+    assert llsa.attn_paths(p)["bwd"] == "tensor"
+    run = GpuRun(case)
+    check_selects_everything(run)
+    check_transpose(run)
+    N = case.H * case.W
+    ref = oracle.dense_attention(run.qh, run.kh, run.vh, run.p.scale, dO=run.gh, keys=np.arange(N))
+    assert_close("O dense", run.o, ref["o"], "bf16")
+    assert_close("LSE dense", run.lse, ref["lse"], "bf16")
+    assert_close("dQ dense", run.dq, ref["dq"], "bf16")
+    assert_close("dK dense", run.dk, ref["dk"], "bf16")
+    assert_close("dV dense", run.dv, ref["dv"], "bf16")
+    if case.H == 64:   # and the loop oracle, fed the (complete) lists
+        check_attention(run, backward=True)
+
+
+def test_dense_bf16_full_size_sampled():
+    """The 256 x 256 workload with K = all and no enrichment against dense
+    attention: O, LSE and dQ on 256 seeded rows of every slice, dK and dV on
+    256 seeded keys of the first slice, the gradient sums on every slice."""
+    from hierarchical_top_sparse_b200 import llsa
+    c = synthetic.CONFIGS["px256"]
+    case = Case(batch=c["batch"], heads=c["heads"], H=c["H"], W=c["W"], L=c["L"], K=10 ** 6, sigma=c["sigma"],
+                enrich_mask=0)
+    p, op = case.problems()
+    assert llsa.attn_paths(p)["bwd"] == "tensor"
+    run = GpuRun(case)
+    check_selects_everything(run)
+    rows = sampled_rows(op.N, 256, 5)
+    ref = oracle.dense_attention(run.qh, run.kh, run.vh, run.p.scale, dO=run.gh, rows=rows)
+    assert_close("O dense rows", run.o[:, rows], ref["o"], "bf16")
+    assert_close("LSE dense rows", run.lse[:, rows], ref["lse"], "bf16")
+    assert_close("dQ dense rows", run.dq[:, rows], ref["dq"], "bf16")
+    keys = sampled_rows(op.N, 256, 6)
+    ref0 = oracle.dense_attention(run.qh[:1], run.kh[:1], run.vh[:1], run.p.scale, dO=run.gh[:1], rows=rows[:8],
+                                  keys=keys)
+    assert_close("dK dense keys", run.dk[:1, keys], ref0["dk"], "bf16")
+    assert_close("dV dense keys", run.dv[:1, keys], ref0["dv"], "bf16")
+    check_gradient_sums(run)
+
+
 def test_select_and_transpose_are_deterministic():
     case = Case(batch=2, heads=2, H=64, W=64, L=3, K=8)
     a, b = GpuRun(case), GpuRun(case)
@@ -171,7 +273,7 @@ def test_workload_128(cfg):
     if c["backward"]:
         check_transpose(run)
     check_attention(run, backward=c["backward"])
-    check_end_to_end(run)
+    check_end_to_end(run, grads=c["backward"])
     print(f"{cfg}: {ties} near-tie rows")
 
 
@@ -180,7 +282,7 @@ def sampled_rows(N, count, seed):
     return np.sort(rng.choice(N, size=count, replace=False))
 
 
-@pytest.mark.parametrize("cfg,full_slices", [("px256", (0, 7)), ("px512", ())])
+@pytest.mark.parametrize("cfg,full_slices", [("px256", (0, 7)), ("px512", (0,))])
 def test_workload_full_size(cfg, full_slices):
     """The full-size workloads in the launch configuration the benchmark times:
     every selection level and the transposes in full, O / LSE / dQ on sampled
@@ -200,11 +302,71 @@ def test_workload_full_size(cfg, full_slices):
     assert_close("LSE rows", run.lse[:, rows], lse[:, rows], "bf16")
     dq = oracle.attn_dq_rows(op, run.qh, run.kh, run.vh, pk, pv, run.idx, run.gh, rows)
     assert_close("dQ rows", run.dq[:, rows], dq[:, rows], "bf16")
-    # sum_t dV_t = sum_i dO_i and sum_t dK_t = 0, per slice and channel
+    check_gradient_sums(run)
+    for s in full_slices:
+        check_attention(run, backward=True, sel=slice(s, s + 1))
+    # end to end (the oracle's own selection): O and LSE on every slice, the
+    # gradients on the first
+    check_end_to_end(run, grads=False)
+    check_end_to_end(run, sel=slice(0, 1))
+
+
+def check_gradient_sums(run: GpuRun):
+    # every row's softmax weights sum to one and its dS to zero: sum_t dV_t =
+    # sum_i dO_i and sum_t dK_t = 0, per slice and channel
     sv = run.dv.astype(np.float64).sum(axis=1)
     np.testing.assert_allclose(sv, run.gh.astype(np.float64).sum(axis=1), rtol=0, atol=0.5 + 2e-3 * np.abs(sv).max())
     sk = run.dk.astype(np.float64).sum(axis=1)
     scale_k = np.abs(run.dk).sum(axis=1)
     assert np.all(np.abs(sk) <= 2e-2 * scale_k + 1e-3), "sum of dK is not ~0"
-    for s in full_slices:
-        check_attention(run, backward=True, sel=slice(s, s + 1))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_level1_pyramid_contract(dtype):
+    """Level 1 of pyrK / pyrV must be llsa_pool's output for the same K / V.
+    The tensor-core kernels (bf16, d = 64, B = 16) derive level-1 pooled
+    tokens from K and V and never read that level: a perturbed level 1 leaves
+    every output bit unchanged.  The CUDA-core kernels (fp32 here) read it:
+    their outputs follow the oracle fed the perturbed pyramid."""
+    from hierarchical_top_sparse_b200 import llsa
+    case = Case(batch=1, heads=2, H=64, W=64, L=3, K=8, dtype=dtype)
+    p, op = case.problems()
+    tc = llsa.attn_paths(p)
+    assert tc == ({"fwd": "tensor", "bwd": "tensor"} if dtype == "bf16" else {"fwd": "cuda-core", "bwd": "cuda-core"})
+    base = GpuRun(case)
+    pipe = base.pipe
+    qd, kd, vd, gd = (to_dev(x, dtype == "bf16") for x in (base.qh, base.kh, base.vh, base.gh))
+    lvK = llsa.level_views(p, pipe.pyrK, p.d)[0]
+    lvV = llsa.level_views(p, pipe.pyrV, p.d)[0]
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    lvK.add_(0.5 * torch.randn(lvK.shape, device="cuda", generator=gen))
+    lvV.add_(0.5 * torch.randn(lvV.shape, device="cuda", generator=gen))
+    o = torch.empty_like(pipe.o)
+    lse = torch.empty_like(pipe.lse)
+    llsa.attn_fwd(p, qd, kd, vd, pipe.pyrK, pipe.pyrV, pipe.idx, o, lse)
+    dq, dk, dv = torch.empty_like(pipe.dq), torch.empty_like(pipe.dk), torch.empty_like(pipe.dv)
+    llsa.attn_bwd(p, qd, kd, vd, o, gd, lse, pipe.pyrK, pipe.pyrV, pipe.idx, pipe.offs, pipe.qlist, dq, dk, dv,
+                  pipe.work)
+    torch.cuda.synchronize()
+    assert llsa.device_error() == 0
+    shape = (p.BH, p.N, p.d)
+    got = {"o": to_np(o).reshape(shape), "lse": to_np(lse).reshape(p.BH, p.N), "dq": to_np(dq).reshape(shape),
+           "dk": to_np(dk).reshape(shape), "dv": to_np(dv).reshape(shape)}
+    if dtype == "bf16":
+        # O, LSE and dQ are deterministic: bit for bit.  dK and dV add the
+        # pooled-key gradients, summed with fp32 atomics in arbitrary order:
+        # within one bf16 rounding step of the unperturbed run (the 0.5
+        # perturbation would move them by far more if level 1 were read).
+        for name in ("o", "lse", "dq"):
+            np.testing.assert_array_equal(got[name], getattr(base, name), err_msg=f"{name} read level 1")
+        for name in ("dk", "dv"):
+            ref = getattr(base, name)
+            assert np.all(np.abs(got[name] - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-6), f"{name} read level 1"
+        return
+    pk = [t.cpu().numpy().astype(np.float64) for t in llsa.level_views(p, pipe.pyrK, p.d)]
+    pv = [t.cpu().numpy().astype(np.float64) for t in llsa.level_views(p, pipe.pyrV, p.d)]
+    ro, rlse = oracle.attn_fwd(op, base.qh, base.kh, base.vh, pk, pv, base.idx)
+    rdq, rdk, rdv, _, _ = oracle.attn_bwd(op, base.qh, base.kh, base.vh, pk, pv, base.idx, base.gh)
+    assert errors(got["o"], base.o)[0] > 1e-3, "the perturbation did not reach the output"
+    for name, want in (("o", ro), ("lse", rlse), ("dq", rdq), ("dk", rdk), ("dv", rdv)):
+        assert_close(name + " (perturbed level 1)", got[name], want, dtype)

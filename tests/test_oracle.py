@@ -406,3 +406,29 @@ def test_single_level_backward_matches_finite_differences():
             fd = (_loss(p, plus["q"], plus["k"], plus["v"], idx, g)
                   - _loss(p, minus["q"], minus["k"], minus["v"], idx, g)) / (2 * h)
             assert abs(fd - grad[0, t, c]) <= 1e-6 * max(1.0, abs(fd)), (which, t, c, fd, grad[0, t, c])
+
+
+def test_dense_reference_matches_autograd_on_row_and_key_subsets():
+    # the closed form the K = all mode is compared with on the GPU: pinned
+    # against torch autograd of softmax(q k^T s) v, and against the loop
+    # oracle at K = all without enrichment
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(11)
+    p = oracle.Problem(H=16, W=16, d=8, B=16, L=2, K=10 ** 6, enrich_mask=0)
+    q, k, v, g = (_rand(rng, 2, p.N, p.d) for _ in range(4))
+    rows = np.array([0, 3, 17, 100, 255])
+    keys = np.array([1, 2, 50, 254])
+    ref = oracle.dense_attention(q, k, v, p.scale, dO=g, rows=rows, keys=keys, chunk=64)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    z = tq @ tk.transpose(-1, -2) * p.scale
+    out = torch.softmax(z, dim=-1) @ tv
+    (out * torch.tensor(g)).sum().backward()
+    np.testing.assert_allclose(ref["o"], out.detach().numpy()[:, rows], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ref["lse"], torch.logsumexp(z, -1).detach().numpy()[:, rows], rtol=1e-12)
+    np.testing.assert_allclose(ref["dq"], tq.grad.numpy()[:, rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(ref["dk"], tk.grad.numpy()[:, keys], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(ref["dv"], tv.grad.numpy()[:, keys], rtol=1e-10, atol=1e-12)
+    r = oracle.forward(p, q, k, v)
+    dq, dk, dv, _, _ = oracle.attn_bwd(p, q, k, v, r["pyrK"], r["pyrV"], r["idx"], g)
+    np.testing.assert_allclose(ref["o"], r["o"][:, rows], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(ref["dk"], dk[:, keys], rtol=1e-10, atol=1e-12)
