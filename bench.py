@@ -273,7 +273,7 @@ def traffic_record(kernel_stage: str):
 
 # The sources each stage's kernels are built from (the shared headers included).
 STAGE_SOURCES = {
-    "attn_fwd": ("k_attn_fwd_mma.cu",),
+    "attn_fwd": ("k_attn_fwd_tc.cu",),
     "attn_bwd": ("k_attn_bwd.cu", "k_attn_bwd_q_tc.cu", "k_attn_bwd_kv_tc.cu"),
 }
 SHARED_HEADERS = ("llsa_internal.cuh", "ptx.cuh", "tcgen05.cuh")

@@ -29,9 +29,11 @@
 // pairs, computed and discarded.
 //
 // Warp roles, one CTA per SM (22 warps):
-//   * warp 20, producer: takes the CTA's key groups (grid stride, so that the
-//     CTAs in flight share neighbouring Q/dO tiles in L2), reads each group's
-//     union (prefetched two groups ahead), and loads every chunk (one lane
+//   * warp 20, producer: claims key groups one at a time from a counter that
+//     all CTAs share (the CTAs in flight then work on neighbouring groups and
+//     share their Q/dO tiles in L2, and a CTA that drew long unions does not
+//     hold up the launch), reads each group's union (prefetched one group
+//     ahead), and loads every chunk (one lane
 //     per 2 KB tile) into one of NSLOT slots and every group's K and V (one
 //     16 KB box each) into one of two key slots, all with TMA;
 //   * warp 21, MMA: a converged warp whose elected lane issues the MMAs and
@@ -39,8 +41,9 @@
 //   * warps 0-15, softmax: warps w, w + 4, w + 8, w + 12 share TMEM lanes
 //     32 (w % 4).. and take key blocks 2 (w / 4) and 2 (w / 4) + 1 of those
 //     query rows;
-//   * warps 16-19, epilogue: walks the CTA's key groups in the same order
-//     and takes each group's accumulators when the MMA warp hands them over.
+//   * warps 16-19, epilogue: takes the CTA's key groups in claim order from
+//     the producer and each group's accumulators when the MMA warp hands them
+//     over.
 // Every hand-off is an mbarrier, every wait is bounded; on a timeout the
 // kernel sets the device error word and stops.
 //
@@ -73,6 +76,7 @@ constexpr int kLast = 1, kFirst = 2;
 enum : int { kEnd = 0, kChunk = 1 };
 // arrivals that free a chunk slot: the MMA thread and each softmax warp
 constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS;
+constexpr int GRING = 4;            // key-group ids in flight between the producer and the epilogue
 
 struct ChunkSlot {
   alignas(1024) unsigned char q[CQ * 2048];    // [128 queries][64] bf16, 128-byte swizzle
@@ -104,7 +108,9 @@ struct Smem {
   uint64_t s_full, s_empty;                    // S / dP in TMEM: MMA -> softmax, softmax (8 warps) -> MMA
   uint64_t p_full, p_empty;                    // P / dS operands: softmax (8 warps) -> MMA, MMA -> softmax
   uint64_t acc_full[2], acc_empty[2];          // accumulator buffers: MMA -> epilogue, epilogue (4 warps) -> MMA
+  uint64_t gid_full[GRING], gid_empty[GRING];  // the CTA's key groups in claim order: producer -> epilogue
   uint64_t drain;
+  int gid[GRING];
   uint32_t tmem_base;
 };
 
@@ -121,7 +127,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo, const float* __restrict__ lse,
     const float* __restrict__ Dws, const int32_t* __restrict__ offs, const int32_t* __restrict__ ulist,
     const int32_t* __restrict__ ucount, const float* __restrict__ dPK, const float* __restrict__ dPV,
-    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int* err) {
+    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int* __restrict__ counter, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,6 +151,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&s.acc_full[i], 1);
       ptx::mbar_init(&s.acc_empty[i], 4);
+    }
+    for (int i = 0; i < GRING; ++i) {
+      ptx::mbar_init(&s.gid_full[i], 1);
+      ptx::mbar_init(&s.gid_empty[i], 4);
     }
     ptx::mbar_init(&s.drain, 1);
     ptx::fence_mbar_init();
@@ -224,16 +234,24 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       ++issued;
     };
 
-    // Group k of this CTA is blockIdx.x + k * gridDim.x.  Lane 0 holds the
-    // start and size of a group's union; all lanes hold its first 64 entries.
-    const int stride = (int)gridDim.x;
-    auto info = [&](int gi, int& lo, int& cnt) {   // issues the loads only
-      lo = cnt = 0;
+    // Key groups are claimed one at a time from a counter shared by all
+    // CTAs (so that a CTA that drew long unions does not hold up the launch),
+    // one group ahead of the one being loaded.  Lane 0 holds the start and
+    // size of a group's union; all lanes hold its first 64 entries.
+    auto claim = [&]() -> int {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
+    auto info = [&](int gi, int& lo, int& cnt) {
+      int a = 0, b = 0;
       if (gi < ngroups && lane == 0) {
         const int bh = gi * KG / n1;
-        lo = offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + (gi * KG - bh * n1)];
-        cnt = ucount[gi];
+        a = offs[g.offs_off[1] + (int64_t)bh * (n1 + 1) + (gi * KG - bh * n1)];
+        b = ucount[gi];
       }
+      lo = __shfl_sync(0xffffffffu, a, 0);
+      cnt = __shfl_sync(0xffffffffu, b, 0);
     };
     auto entries = [&](int gi, int lo, int cnt, int& e0, int& e1) {
       e0 = e1 = 0;
@@ -243,28 +261,30 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         if (32 + lane < cnt) e1 = ul[32 + lane];
       }
     };
-    int gi = (int)blockIdx.x;
-    int lo_c = 0, cnt_c = 0, e0c = 0, e1c = 0;       // group k
-    int lo_n = 0, cnt_n = 0, e0n = 0, e1n = 0;       // group k + 1
-    int lo_nn = 0, cnt_nn = 0;                       // group k + 2 (lane 0)
-    {
-      int a, b;
-      info(gi, a, b);
-      lo_n = __shfl_sync(0xffffffffu, a, 0);
-      cnt_n = __shfl_sync(0xffffffffu, b, 0);
-      entries(gi, lo_n, cnt_n, e0n, e1n);
-      info(gi + stride, lo_nn, cnt_nn);
-    }
-    for (; gi < ngroups && ok; gi += stride) {
-      // rotate the prefetch pipeline
-      lo_c = lo_n;
-      cnt_c = cnt_n;
-      e0c = e0n;
-      e1c = e1n;
-      lo_n = __shfl_sync(0xffffffffu, lo_nn, 0);
-      cnt_n = __shfl_sync(0xffffffffu, cnt_nn, 0);
-      entries(gi + stride, lo_n, cnt_n, e0n, e1n);
-      info(gi + 2 * stride, lo_nn, cnt_nn);
+    // hands the group id (or -1: no more) to the epilogue, in claim order
+    uint32_t gcount = 0;
+    auto announce = [&](int gi) {
+      const int r = (int)(gcount % GRING);
+      wait_free(&s.gid_empty[r], ((gcount / GRING) & 1) ^ 1, 40);
+      if (!ok) return;
+      if (lane == 0) {
+        s.gid[r] = gi;
+        ptx::mbar_arrive(&s.gid_full[r]);
+      }
+      __syncwarp();
+      ++gcount;
+    };
+    int gi = claim();
+    int lo_n = 0, cnt_n = 0, e0n = 0, e1n = 0;
+    info(gi, lo_n, cnt_n);
+    entries(gi, lo_n, cnt_n, e0n, e1n);
+    while (gi < ngroups && ok) {
+      const int lo_c = lo_n, cnt_c = cnt_n, e0c = e0n, e1c = e1n;
+      const int gnext = claim();     // prefetch the next group's union while this one streams
+      info(gnext, lo_n, cnt_n);
+      entries(gnext, lo_n, cnt_n, e0n, e1n);
+      announce(gi);
+      if (!ok) break;
 
       const int kbg0 = gi * KG;
       const int64_t bh = kbg0 / n1;
@@ -294,7 +314,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         const int flags = (c == 0 ? kFirst : 0) | (c == nchunks - 1 ? kLast : 0);
         emit(kbg0, bh, nq > 0 ? nq : 0, flags, e >> 8, e & 0xff);
       }
+      gi = gnext;
     }
+    if (ok) announce(-1);
     if (ok) {   // the end marker: every consumer leaves its loop on it
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 43);
@@ -562,8 +584,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const int sub = warp & 3;
     const int row = sub * 32 + lane;                    // key of the group (TMEM lane)
     const uint32_t tl = tbase + ((uint32_t)(sub * 32) << 16);
-    uint32_t k = 0;
-    for (int gi = (int)blockIdx.x; gi < ngroups; gi += (int)gridDim.x, ++k) {
+    for (uint32_t k = 0;; ++k) {
+      const int r = (int)(k % GRING);
+      if (!ptx::mbar_wait_bounded(&s.gid_full[r], (k / GRING) & 1, kWaitLimitNs)) {
+        report(err, 47);
+        break;
+      }
+      const int gi = s.gid[r];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.gid_empty[r]);
+      if (gi < 0) break;
       const int kbg0 = gi * KG;
       const int bh = kbg0 / n1;
       const int64_t t0 = (int64_t)(kbg0 - bh * n1) * 16;   // the group's first key within its slice
@@ -648,7 +678,7 @@ cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, co
   const int grid = ngroups < sms ? ngroups : sms;
   bwdtc::attn_bwd_kv_tc_kernel<<<grid, bwdtc::THREADS, smem, s>>>(g, tk, tv, tq, tdo, lse, ws.D, offs, ws.ulist_kv,
                                                                    ws.ucount_kv, ws.dPK, ws.dPV, (__nv_bfloat16*)dk,
-                                                                   (__nv_bfloat16*)dv, device_error_word());
+                                                                   (__nv_bfloat16*)dv, ws.counter, device_error_word());
   note_launches(1);
   return cudaGetLastError();
 }

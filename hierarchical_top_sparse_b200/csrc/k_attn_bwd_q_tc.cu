@@ -29,7 +29,8 @@
 // the swizzled operand layout, bias, level, id).
 //
 // Warp roles of the main kernel, one CTA per SM (22 warps):
-//   * warp 20, producer: walks the CTA's tokens (grid stride), loads each
+//   * warp 20, producer: claims tokens one at a time from a counter that all
+//     CTAs share (and hands their ids to the epilogue warps), loads each
 //     group's Q and dO (one 128-row TMA box each) into one of two group
 //     slots, the token's pooled-key tile (one bulk copy) into one of two
 //     coarse slots, and the K/V tiles of each union chunk (one lane per 2 KB
@@ -71,6 +72,7 @@ constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_DS = 320, COL_GK =
 enum : int { kEnd = 0, kChunk = 1, kTail = 2 };
 constexpr int kFirst = 1;           // first entry of a group
 constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS;   // a chunk slot is freed by the MMA thread and every softmax warp
+constexpr int TRING = 4;            // token ids in flight between the producer and the epilogue
 
 struct ChunkSlot {
   alignas(1024) unsigned char k[CK * 2048];    // [128 keys][64] bf16, 128-byte swizzle
@@ -121,7 +123,9 @@ struct Smem {
   uint64_t p_full, p_empty;                    // dS operand: softmax (16 warps) -> MMA, MMA -> softmax
   uint64_t acc_full, acc_empty;                // dQ of a group (phase = the CTA's group count): MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t cacc_full, cacc_empty;              // pooled-key gradients: MMA -> epilogue, epilogue (4 warps) -> MMA
+  uint64_t tid_full[TRING], tid_empty[TRING];  // the CTA's tokens in claim order: producer -> epilogue
   uint64_t drain;
+  int tid[TRING];
   uint32_t tmem_base;
 };
 
@@ -341,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, const float* __restrict__ lse,
     const float* __restrict__ Dws, const int32_t* __restrict__ ulist, const int32_t* __restrict__ ucount,
     const unsigned char* __restrict__ ctile, __nv_bfloat16* __restrict__ dq, float* __restrict__ dPK,
-    float* __restrict__ dPV, int* err) {
+    float* __restrict__ dPV, int* __restrict__ counter, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -371,6 +375,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     ptx::mbar_init(&s.acc_empty, 4);
     ptx::mbar_init(&s.cacc_full, 1);
     ptx::mbar_init(&s.cacc_empty, 4);
+    for (int i = 0; i < TRING; ++i) {
+      ptx::mbar_init(&s.tid_full[i], 1);
+      ptx::mbar_init(&s.tid_empty[i], 4);
+    }
     ptx::mbar_init(&s.drain, 1);
     ptx::fence_mbar_init();
   }
@@ -451,8 +459,27 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       ++issued;
     };
 
+    // Tokens are claimed one at a time from a counter that all CTAs share,
+    // and handed to the epilogue warps in claim order (-1: no more).
+    auto announce = [&](uint32_t k, int t) {
+      const int r = (int)(k % TRING);
+      wait_free(&s.tid_empty[r], ((k / TRING) & 1) ^ 1, 50);
+      if (!ok) return;
+      if (lane == 0) {
+        s.tid[r] = t;
+        ptx::mbar_arrive(&s.tid_full[r]);
+      }
+      __syncwarp();
+    };
+    auto claim = [&]() -> int {
+      int v = 0;
+      if (lane == 0) v = atomicAdd(counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
     uint32_t tk_n = 0;   // tokens done by this CTA
-    for (int t = (int)blockIdx.x; t < ntokens && ok; t += stride, ++tk_n) {
+    for (int t = claim(); t < ntokens && ok; t = claim(), ++tk_n) {
+      announce(tk_n, t);
+      if (!ok) break;
       // the token's two groups: counts and first 64 union entries, then Q / dO
       int cnt[2], e0[2], e1[2];
 #pragma unroll
@@ -508,6 +535,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
         if (gs == 0 && nchunks == 0 && ok) load_group(1);
       }
     }
+    if (ok) announce(tk_n, -1);
     if (ok) {   // the end marker: the MMA and softmax warps leave their loops on it
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 53);
@@ -946,8 +974,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       }
     };
 
-    uint32_t tk = 0;
-    for (int t = (int)blockIdx.x; t < ntokens && ok; t += stride, ++tk) {
+    for (uint32_t tk = 0; ok; ++tk) {
+      const int r = (int)(tk % TRING);
+      if (!ptx::mbar_wait_bounded(&s.tid_full[r], (tk / TRING) & 1, kWaitLimitNs)) {
+        fail(63);
+        break;
+      }
+      const int t = s.tid[r];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&s.tid_empty[r]);
+      if (t < 0) break;
       store_dq(t, tk, 0);
       if (ok) store_dq(t, tk, 1);
       if (ok && nc > 0) coarse_grads(t, tk);
@@ -1002,7 +1038,7 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   const int grid = ntokens < sms ? ntokens : sms;
   bwdq::attn_bwd_q_tc_kernel<<<grid, bwdq::THREADS, smem, s>>>(g, tq128, tdo128, tk, tv, lse, ws.D, ws.ulist,
                                                                 ws.ucount, ws.ctile, (__nv_bfloat16*)dq, ws.dPK,
-                                                                ws.dPV, device_error_word());
+                                                                ws.dPV, ws.counter + 1, device_error_word());
   note_launches(1);
   return cudaGetLastError();
 }

@@ -96,7 +96,8 @@ cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows,
 constexpr int kSelectMaxCandidates = 24576;   // 192 KB of 64-bit keys, one warp
 
 // Workspace of the backward pass: D [BH][N] fp32, the fp32 level gradients
-// of the pooled K and of the pooled V (each a pyramid), a work counter, then
+// of the pooled K and of the pooled V (each a pyramid), two work counters
+// (key groups claimed by the key-major pass, tokens by the query-major pass), then
 // the query groups' unions (each entry block << 8 | pick mask, laid out like
 // the level-1 index lists) and their sizes, one tile of the pooled keys of
 // levels >= 2 per level-2 token (kBwdCoarseTileBytes each), then the key
@@ -111,7 +112,7 @@ struct BwdWorkspace {
   unsigned char* ctile;
   int32_t* ulist_kv;
   int32_t* ucount_kv;
-  size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counter)
+  size_t zero_bytes;   // bytes from dPK on that must start at zero (sums and counters)
 };
 
 // A level-2 token's pooled keys of levels >= 2 (at most 32): K and V rows as
@@ -149,7 +150,7 @@ inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
                       reinterpret_cast<unsigned char*>(after + usz + csz),
                       reinterpret_cast<int32_t*>(kv),
                       reinterpret_cast<int32_t*>(kv + usz),
-                      2 * pyr + sizeof(int)};
+                      2 * pyr + 2 * sizeof(int)};
 }
 
 // ------------------------------------------------------------ device helpers

@@ -50,6 +50,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, letting the hardware suspend the thread until the phase
+// completes or about `hint_ns` pass, so that a waiting warp takes neither
+// issue slots nor shared-memory barrier bandwidth from the warps at work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -58,14 +75,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // The slow part of a bounded wait, kept out of line and not unrolled: every
 // wait site inlines only its first test, so that the kernels' code stays
-// small enough for the instruction caches.
+// small enough for the instruction caches.  The thread sleeps in the
+// barrier (woken when the phase completes) rather than polling it, in steps
+// short against the limit.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
+  const uint32_t step = limit_ns < 8000000ull ? (uint32_t)(limit_ns / 8 + 1) : 1000000u;
 #pragma unroll 1
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, step)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }

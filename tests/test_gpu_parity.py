@@ -215,7 +215,7 @@ def test_dense_bf16_on_the_tensor_cores(name):
     from hierarchical_top_sparse_b200 import llsa
     case = DENSE_BF16[name]
     p, _ = case.problems()
-    assert llsa.attn_paths(p)["bwd"] == "tensor"
+    assert llsa.attn_paths(p) == {"fwd": "tensor", "bwd": "tensor"}
     run = GpuRun(case)
     check_selects_everything(run)
     check_transpose(run)
@@ -239,7 +239,7 @@ def test_dense_bf16_full_size_sampled():
     case = Case(batch=c["batch"], heads=c["heads"], H=c["H"], W=c["W"], L=c["L"], K=10 ** 6, sigma=c["sigma"],
                 enrich_mask=0)
     p, op = case.problems()
-    assert llsa.attn_paths(p)["bwd"] == "tensor"
+    assert llsa.attn_paths(p) == {"fwd": "tensor", "bwd": "tensor"}
     run = GpuRun(case)
     check_selects_everything(run)
     rows = sampled_rows(op.N, 256, 5)
