@@ -77,7 +77,7 @@ constexpr int QG = 8;               // query blocks per group (128 queries)
 constexpr int CK = 8;               // key blocks per chunk (128 keys)
 constexpr int NSLOT = 4;            // K / V chunk slots
 constexpr int NQ = 3;               // Q slots: the next group's Q lands while the last two finish
-constexpr int NMETA = 8;            // entries in flight between the union warp and the others
+constexpr int NMETA = 16;           // entries in flight between the union warp and the others
 constexpr int COARSE = 32;          // pooled keys of levels >= 2 per token, at most
 constexpr int STAGE = 512;          // pick-list words a group stages in shared memory
 constexpr int RUNMAX = 4;           // key blocks one TMA box may carry (tensor maps of 16, 32, 48, 64 rows)
@@ -557,8 +557,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
     // ============================================================ MMA issue
     // Converged warp, one elected lane issues.  Descriptors are built once and
     // advanced by adding to their start-address field (16-byte units, no
-    // carry: shared addresses are below 256 KB).  An entry's ring slot is
-    // released once its O update is issued.
+    // carry: shared addresses are below 256 KB).
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S: A = Q (K-major), B = K (K-major)
     constexpr uint32_t idSc = tc::idesc_bf16(128, 32, 0, 0);   // the same against the 32 pooled keys
     constexpr uint32_t idO = tc::idesc_bf16(128, 64, 0, 1);    // O += P V: A = P (TMEM), B = V (MN-major)
@@ -571,7 +570,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
     const uint64_t dcv0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].v), 16, 1024);
     bool ok = true;
     uint32_t seen = 0, sidx = 0;
-    struct Entry { int kind, nq, ms; uint32_t gc, tk, kc, sb; };
+    struct Entry { int kind, nq; uint32_t gc, tk, kc, sb; int msk[CK]; };
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok && !ptx::mbar_wait_bounded(bar, parity, kWaitLimitNs)) ok = false;
       return ok;
@@ -583,11 +582,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       const Meta& m = s.meta[ms];
       c.kind = m.kind;
       c.nq = m.nq;
-      c.ms = ms;
       c.gc = (uint32_t)m.gc;
       c.tk = (uint32_t)m.tk;
       c.kc = (uint32_t)m.kc;
+#pragma unroll
+      for (int j = 0; j < CK; ++j) c.msk[j] = m.msk[j];
       const int flags = m.flags;
+      __syncwarp();
+      if (tc::elect_one()) ptx::mbar_arrive(&s.mempty[ms]);   // the entry is in registers
+      __syncwarp();
       ++seen;
       if (c.kind == kEnd) return false;
       const uint32_t qs = c.gc % NQ;
@@ -627,7 +630,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
     auto finish = [&](const Entry& c) {
       const uint32_t ob = c.gc & 1;
       const bool chunk = c.kind == kChunk && c.nq > 0;
-      const Meta& m = s.meta[c.ms];
       if (c.kind == kCoarse || chunk) {
         const uint32_t b = c.sb & 1, u = c.sb >> 1;
         if (!wait(&s.p_full[b], u & 1)) return;
@@ -642,7 +644,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
             for (int k = 0; k < CK; ++k) {   // key block k: A 8 TMEM columns, B 2 KB
               if (k >= c.nq) break;
               // rows of the query blocks that did not pick block k keep their O
-              const unsigned skip = ~(unsigned)m.msk[k] & 0xffu;
+              const unsigned skip = ~(unsigned)c.msk[k] & 0xffu;
               uint32_t off[4];
 #pragma unroll
               for (int w = 0; w < 4; ++w)
@@ -670,8 +672,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
         __syncwarp();
         o_started = false;
       }
-      if (tc::elect_one()) ptx::mbar_arrive(&s.mempty[c.ms]);   // the entry's ring slot is free
-      __syncwarp();
     };
 
     Entry cur;

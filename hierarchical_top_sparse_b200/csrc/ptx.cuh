@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tensor
-// loads, ldmatrix / mma.sync fragments, and a bounded wait.
+// loads, a bounded wait, and a few arithmetic helpers.
 #pragma once
 
 #include <cuda.h>
@@ -50,23 +50,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// The same test, letting the hardware suspend the thread until the phase
-// completes or about `hint_ns` pass, so that a waiting warp takes neither
-// issue slots nor shared-memory barrier bandwidth from the warps at work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n"
-      ".reg .pred p;\n"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-      "selp.u32 %0, 1, 0, p;\n"
-      "}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -75,15 +58,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // The slow part of a bounded wait, kept out of line and not unrolled: every
 // wait site inlines only its first test, so that the kernels' code stays
-// small enough for the instruction caches.  The thread sleeps in the
-// barrier (woken when the phase completes) rather than polling it, in steps
-// short against the limit.
+// small enough for the instruction caches.  (Polling: letting the thread
+// sleep in the barrier between tests measured slower.)
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
-  const uint32_t step = limit_ns < 8000000ull ? (uint32_t)(limit_ns / 8 + 1) : 1000000u;
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, step)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
@@ -93,34 +76,6 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, limit_ns);
-}
-
-// Release store / acquire load of a shared-memory word (CTA scope).
-__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-
-static __device__ __noinline__ bool wait_u32_equal_slow(const uint32_t* p, uint32_t want, uint64_t limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-#pragma unroll 1
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (ld_acquire_u32(p) == want) return true;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-}
-
-// Waits until the shared word equals `want`, at most `limit_ns` of wall time.
-__device__ __forceinline__ bool wait_u32_equal(const uint32_t* p, uint32_t want, uint64_t limit_ns) {
-  if (ld_acquire_u32(p) == want) return true;
-  return wait_u32_equal_slow(p, want, limit_ns);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -154,38 +109,11 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// ------------------------------------------------------- warp-level MMA
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                                  uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
-__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Byte offset of element (row, col) of a [rows][64] bf16 tile stored with the
-// 128-byte TMA swizzle (16-byte chunk c of row r sits at chunk c ^ (r & 7));
-// the tile must start on a 1024-byte boundary.
 // 2^x by the PTX approximate base-2 exponential (ex2.approx.ftz.f32: a few ulp
 // of relative error, results below 2^-126 flushed to zero, 2^-inf = 0).  The
 // softmax weights it produces are rounded to bf16 right after.
@@ -201,6 +129,9 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
+// Byte offset of element (row, col) of a [rows][64] bf16 tile stored with the
+// 128-byte TMA swizzle (16-byte chunk c of row r sits at chunk c ^ (r & 7));
+// the tile must start on a 1024-byte boundary.
 __device__ __forceinline__ uint32_t sw128(int row, int col) {
   return (uint32_t)(row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1));
 }
