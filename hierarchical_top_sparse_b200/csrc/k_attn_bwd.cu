@@ -48,9 +48,9 @@ cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const int32_t* idx, const int32_t* offs, const int32_t* qlist, void* dq, void* dk,
                                 void* dv, void* workspace, cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
-  CUtensorMap tq, tdo;   // 16-row boxes: the key-major pass stacks query blocks
-  cudaError_t e = make_token_map(&tq, q, rows);
-  if (e == cudaSuccess) e = make_token_map(&tdo, dO, rows);
+  RunMaps tq, tdo;   // boxes of 1..4 query blocks: the key-major pass stacks them
+  cudaError_t e = make_run_maps(&tq, q, rows);
+  if (e == cudaSuccess) e = make_run_maps(&tdo, dO, rows);
   if (e != cudaSuccess) return e;
   BwdWorkspace ws = carve_bwd_workspace(g, workspace);
   e = cudaMemsetAsync(ws.dPK, 0, ws.zero_bytes, s);   // pooled-key sums and the work counter

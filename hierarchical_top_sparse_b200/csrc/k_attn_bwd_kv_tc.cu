@@ -124,7 +124,7 @@ __device__ __forceinline__ void report(int* err, int code) {
 
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const __grid_constant__ Geo g, const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-    const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo, const float* __restrict__ lse,
+    const __grid_constant__ RunMaps tq, const __grid_constant__ RunMaps tdo, const float* __restrict__ lse,
     const float* __restrict__ Dws, const int32_t* __restrict__ offs, const int32_t* __restrict__ ulist,
     const int32_t* __restrict__ ucount, const float* __restrict__ dPK, const float* __restrict__ dPV,
     __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int* __restrict__ counter, int* err) {
@@ -181,8 +181,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     if (lane == 0) {
       ptx::prefetch_tmap(&tk);
       ptx::prefetch_tmap(&tv);
-      ptx::prefetch_tmap(&tq);
-      ptx::prefetch_tmap(&tdo);
+    }
+    if (lane < kRunMax) {
+      ptx::prefetch_tmap(&tq.m[lane]);
+      ptx::prefetch_tmap(&tdo.m[lane]);
     }
     uint32_t issued = 0, kissued = 0;
     bool ok = true;
@@ -196,7 +198,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       }
     };
     // One chunk of nq query blocks of the group at kbg0 (lane j < nq holds
-    // member j in pq / pm): lane j loads its Q tile, lane 8 + j its dO tile.
+    // member j in pq / pm).  A run of consecutive query blocks is one box of
+    // up to four tiles: lane j issues the Q box that starts at member j, lane
+    // 8 + j the dO box.
     auto emit = [&](int kbg0, int64_t bh, int nq, int flags, int pq, int pm) {
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 41);
@@ -222,13 +226,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       __syncwarp();
       const int j = lane & 7;
       const int qj = __shfl_sync(0xffffffffu, pq, j);
-      if (lane < 16 && j < nq) {
+      const int box = __shfl_sync(0xffffffffu, run_box(pq, nq, lane), j);
+      if (lane < 16 && box > 0) {
         const int row = (int)((bh * n1 + qj) * 16);
         ChunkSlot& cs = s.slot[slot];
         if (lane < 8)
-          ptx::tma_load_2d(cs.q + j * 2048, &tq, 0, row, bar);
+          ptx::tma_load_2d(cs.q + j * 2048, &tq.m[box - 1], 0, row, bar);
         else
-          ptx::tma_load_2d(cs.dO + j * 2048, &tdo, 0, row, bar);
+          ptx::tma_load_2d(cs.dO + j * 2048, &tdo.m[box - 1], 0, row, bar);
       }
       __syncwarp();
       ++issued;
@@ -661,8 +666,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
 
 // Needs n_1 to be a multiple of 16 (checked by the caller): key groups of 8
 // blocks never cross a slice and lie under one level-2 token.
-cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
-                                  const CUtensorMap& tdo, const float* lse, const int32_t* offs,
+cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const RunMaps& tq,
+                                  const RunMaps& tdo, const float* lse, const int32_t* offs,
                                   const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s) {
   CUtensorMap tk, tv;   // one box = one key group (8 blocks, 128 rows)
   cudaError_t e = make_token_map_box(&tk, k, (int64_t)g.BH * g.N, bwdtc::KG * 16);

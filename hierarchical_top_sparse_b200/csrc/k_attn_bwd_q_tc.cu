@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(PREP_THREADS) q_prep_kernel(Geo g, const int32
 
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
     const __grid_constant__ Geo g, const __grid_constant__ CUtensorMap tq128, const __grid_constant__ CUtensorMap tdo128,
-    const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, const float* __restrict__ lse,
+    const __grid_constant__ RunMaps tk, const __grid_constant__ RunMaps tv, const float* __restrict__ lse,
     const float* __restrict__ Dws, const int32_t* __restrict__ ulist, const int32_t* __restrict__ ucount,
     const unsigned char* __restrict__ ctile, __nv_bfloat16* __restrict__ dq, float* __restrict__ dPK,
     float* __restrict__ dPV, int* __restrict__ counter, int* err) {
@@ -398,15 +398,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = s.tmem_base;
-  const int stride = (int)gridDim.x;
 
   if (warp == PRODUCER_WARP) {
     // ============================================================ producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tq128);
       ptx::prefetch_tmap(&tdo128);
-      ptx::prefetch_tmap(&tk);
-      ptx::prefetch_tmap(&tv);
+    }
+    if (lane < kRunMax) {
+      ptx::prefetch_tmap(&tk.m[lane]);
+      ptx::prefetch_tmap(&tv.m[lane]);
     }
     uint32_t issued = 0;
     bool ok = true;
@@ -420,8 +421,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       }
     };
     // One ring entry: a chunk of nq key blocks (lane j < nq holds block j and
-    // its mask in ek / em) or a group's closing entry.  Lane j loads block
-    // j's K tile, lane 8 + j its V tile.
+    // its mask in ek / em) or a group's closing entry.  A run of consecutive
+    // key blocks is one box of up to four tiles: lane j issues the K box that
+    // starts at block j, lane 8 + j the V box.
     auto emit = [&](int kind, int gi, int gs, int64_t bh, int nq, int flags, int ek, int em) {
       const int slot = (int)(issued % NSLOT);
       wait_free(&s.empty[slot], ((issued / NSLOT) & 1) ^ 1, 51);
@@ -447,13 +449,14 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_q_tc_kernel(
       __syncwarp();
       const int j = lane & 7;
       const int kj = __shfl_sync(0xffffffffu, ek, j);
-      if (lane < 16 && j < nq) {
+      const int box = __shfl_sync(0xffffffffu, run_box(ek, nq, lane), j);
+      if (lane < 16 && box > 0) {
         const int row = (int)((bh * n1 + kj) * 16);
         ChunkSlot& cs = s.slot[slot];
         if (lane < 8)
-          ptx::tma_load_2d(cs.k + j * 2048, &tk, 0, row, bar);
+          ptx::tma_load_2d(cs.k + j * 2048, &tk.m[box - 1], 0, row, bar);
         else
-          ptx::tma_load_2d(cs.v + j * 2048, &tv, 0, row, bar);
+          ptx::tma_load_2d(cs.v + j * 2048, &tv.m[box - 1], 0, row, bar);
       }
       __syncwarp();
       ++issued;
@@ -1013,11 +1016,12 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
   if (g.d != 64 || g.B != 16 || g.n[1] % (2 * bwdq::QG) || g.Kl[1] < 1 || nc > bwdq::COARSE)
     return cudaErrorInvalidValue;
   const int64_t rows = (int64_t)g.BH * g.N;
-  CUtensorMap tq128, tdo128, tk, tv;
+  CUtensorMap tq128, tdo128;
+  RunMaps tk, tv;
   cudaError_t e = make_token_map_box(&tq128, q, rows, bwdq::QG * 16);
   if (e == cudaSuccess) e = make_token_map_box(&tdo128, dO, rows, bwdq::QG * 16);
-  if (e == cudaSuccess) e = make_token_map(&tk, k, rows);
-  if (e == cudaSuccess) e = make_token_map(&tv, v, rows);
+  if (e == cudaSuccess) e = make_run_maps(&tk, k, rows);
+  if (e == cudaSuccess) e = make_run_maps(&tv, v, rows);
   if (e != cudaSuccess) return e;
   const int ngroups = (int)((int64_t)g.BH * g.n[1] / bwdq::QG);
   const int ntokens = ngroups / 2;

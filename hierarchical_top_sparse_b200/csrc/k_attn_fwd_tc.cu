@@ -80,7 +80,6 @@ constexpr int NQ = 3;               // Q slots: the next group's Q lands while t
 constexpr int NMETA = 16;           // entries in flight between the union warp and the others
 constexpr int COARSE = 32;          // pooled keys of levels >= 2 per token, at most
 constexpr int STAGE = 512;          // pick-list words a group stages in shared memory
-constexpr int RUNMAX = 4;           // key blocks one TMA box may carry (tensor maps of 16, 32, 48, 64 rows)
 constexpr int SOFT_WARPS = 16;      // four per TMEM subpartition, each on two of a chunk's key blocks
 constexpr int PARTS = SOFT_WARPS / 4;
 constexpr int NPROD = 2;            // producer warps, on alternate entries
@@ -108,11 +107,6 @@ struct alignas(1024) CoarseSlot {
   unsigned char k[COARSE * 128];               // [32 pooled keys][64] bf16, 128-byte swizzle
   unsigned char v[COARSE * 128];
   float bias[COARSE];                          // logit bias (log2 domain); -inf: no key
-};
-
-// Tensor maps of one token tensor with boxes of 1..RUNMAX key blocks (16 rows each).
-struct RunMaps {
-  CUtensorMap m[RUNMAX];
 };
 
 struct Meta {                                  // union warp -> producers, MMA and softmax warps
@@ -273,19 +267,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
         return;
       }
       Meta& M = s.meta[ms];
-      const int prevkb = __shfl_up_sync(0xffffffffu, ekb, 1);
-      const bool brk = lane == 0 || ekb != prevkb + 1;
-      const unsigned starts = __ballot_sync(0xffffffffu, lane < nq && brk);
+      const int box = run_box(ekb, nq, lane);
       if (lane < CK) {
-        int box = 0;
-        if (lane < nq) {
-          const int rs = 31 - __clz(starts & ((2u << lane) - 1u));    // start of this block's run
-          if (((lane - rs) % RUNMAX) == 0) {
-            const unsigned later = starts & ~((2u << lane) - 1u);
-            const int rend = later ? __ffs(later) - 1 : nq;           // end of the run
-            box = min(RUNMAX, rend - lane);
-          }
-        }
         const int64_t bh = (int64_t)gi * QG / n1;
         M.msk[lane] = lane < nq ? em : 0;
         M.row[lane] = lane < nq ? (int)((bh * n1 + ekb) * 16) : 0;
@@ -475,7 +458,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
   } else if (warp >= PRODUCER0 && warp < PRODUCER0 + NPROD) {
     // ============================================================ producers
     const int pw = warp - PRODUCER0;
-    if (lane < RUNMAX) {
+    if (lane < kRunMax) {
       ptx::prefetch_tmap(&tk[lane]);
       ptx::prefetch_tmap(&tv[lane]);
     }
@@ -944,12 +927,10 @@ cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, cons
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s) {
   const int64_t rows = (int64_t)g.BH * g.N;
   CUtensorMap tq128;
-  fwdtc::RunMaps km, vm;
+  RunMaps km, vm;
   cudaError_t e = make_token_map_box(&tq128, q, rows, fwdtc::QG * 16);
-  for (int r = 0; r < fwdtc::RUNMAX && e == cudaSuccess; ++r) {
-    e = make_token_map_box(&km.m[r], k, rows, 16 * (r + 1));
-    if (e == cudaSuccess) e = make_token_map_box(&vm.m[r], v, rows, 16 * (r + 1));
-  }
+  if (e == cudaSuccess) e = make_run_maps(&km, k, rows);
+  if (e == cudaSuccess) e = make_run_maps(&vm, v, rows);
   if (e != cudaSuccess) return e;
   const int ntokens = (int)((int64_t)g.BH * g.n[1] / (2 * fwdtc::QG));
   if (ntokens == 0) return cudaSuccess;

@@ -67,6 +67,15 @@ cudaError_t launch_attn_bwd_simt(const Geo& g, const void* q, const void* k, con
 
 struct BwdWorkspace;
 
+// Tensor maps of one token tensor whose boxes carry 1..kRunMax blocks of 16
+// rows (a run of consecutive blocks is then one TMA copy: issuing a copy
+// costs about as much as moving a 2 KB tile).
+constexpr int kRunMax = 4;
+struct RunMaps {
+  CUtensorMap m[kRunMax];
+};
+cudaError_t make_run_maps(RunMaps* maps, const void* base, int64_t rows);
+
 // Tensor-core attention kernels (bf16, d = 64, B = 16).
 bool attn_bwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_bwd_mma(const Geo& g, const void* q, const void* k, const void* v, const void* o,
@@ -79,17 +88,16 @@ cudaError_t launch_attn_bwd_q_tc(const Geo& g, const void* q, const void* k, con
                                  const void* dO, const float* lse, const float* pyrK, const float* pyrV,
                                  const int32_t* idx, const int32_t* offs, const int32_t* qlist,
                                  const BwdWorkspace& ws, void* dq, cudaStream_t s);
-cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const CUtensorMap& tq,
-                                  const CUtensorMap& tdo, const float* lse, const int32_t* offs,
+cudaError_t launch_attn_bwd_kv_tc(const Geo& g, const void* k, const void* v, const RunMaps& tq,
+                                  const RunMaps& tdo, const float* lse, const int32_t* offs,
                                   const BwdWorkspace& ws, void* dk, void* dv, cudaStream_t s);
 bool attn_fwd_mma_supported(const Geo& g);
 cudaError_t launch_attn_fwd_mma(const Geo& g, const void* q, const void* k, const void* v, const float* pyrK,
                                 const float* pyrV, const int32_t* idx, void* o, float* lse, cudaStream_t s);
 
-// TMA descriptor of a [rows][64] bf16 token tensor, boxes of 16 rows x 64
-// columns (one 2 KB key or query block), 128-byte swizzle.
-cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows);
-// Same with boxes of `box_rows` rows (1..256).
+// TMA descriptor of a [rows][64] bf16 token tensor with boxes of `box_rows`
+// rows (1..256) x 64 columns (16 rows: one 2 KB key or query block),
+// 128-byte swizzle.
 cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 // Largest candidate count the selection kernel keeps in shared memory.
@@ -154,6 +162,23 @@ inline BwdWorkspace carve_bwd_workspace(const Geo& g, void* workspace) {
 }
 
 // ------------------------------------------------------------ device helpers
+
+// TMA boxes over a chunk's blocks: lane j < nq holds block id b (ascending
+// over the lanes).  Returns how many blocks (1..kRunMax) the box starting at
+// block j carries -- runs of consecutive ids share a box -- or 0 when block j
+// lies inside an earlier lane's box.  Every lane of the warp calls it.
+__device__ __forceinline__ int run_box(int b, int nq, int lane) {
+  const int prev = __shfl_up_sync(0xffffffffu, b, 1);
+  const bool brk = lane == 0 || b != prev + 1;
+  const unsigned starts = __ballot_sync(0xffffffffu, lane < nq && brk);
+  if (lane >= nq) return 0;
+  const int rs = 31 - __clz(starts & ((2u << lane) - 1u));    // start of the run
+  if ((lane - rs) % kRunMax) return 0;
+  const unsigned later = starts & ~((2u << lane) - 1u);
+  const int rend = later ? __ffs(later) - 1 : nq;              // end of the run
+  return min(kRunMax, rend - lane);
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

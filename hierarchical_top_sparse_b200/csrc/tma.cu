@@ -20,10 +20,6 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-cudaError_t make_token_map(CUtensorMap* map, const void* base, int64_t rows) {
-  return make_token_map_box(map, base, rows, 16);
-}
-
 cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
@@ -36,6 +32,14 @@ cudaError_t make_token_map_box(CUtensorMap* map, const void* base, int64_t rows,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_run_maps(RunMaps* maps, const void* base, int64_t rows) {
+  for (int r = 0; r < kRunMax; ++r) {
+    cudaError_t e = make_token_map_box(&maps->m[r], base, rows, 16 * (r + 1));
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace llsa
