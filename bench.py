@@ -525,6 +525,124 @@ def run_ours(args, rank, local, world, pg):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ N sweep
+#
+# The shape of the pages' speed figures on this GPU: forward tokens/s of the
+# attention against N for LLSA, the single-level top-K baseline and dense
+# attention (the inference kernel speed-up figure), and backward tokens/s
+# against N (the sparse-KV backward figure, expected roughly flat in N).
+# Dense attention is LLSA with K covering every block and no enrichment: its
+# selection is then trivial and only the attention is timed.
+
+SWEEP_SIDES = (64, 128, 256, 512)
+SWEEP_TOKENS = 786432           # batch x heads x N per step at every N (6 heads; 3 at 512^2)
+DENSE_MAX_BLOCKS = 4096         # the tensor-core attention paths take K_1 <= 4096
+
+
+def sweep_problem(llsa, side: int, mode: str):
+    heads = min(6, SWEEP_TOKENS // (side * side))
+    batch = SWEEP_TOKENS // (heads * side * side)
+    L = 4 if side >= 256 else 3
+    if mode == "llsa":
+        return llsa.Problem(batch=batch, heads=heads, height=side, width=side, d=64, B=16, L=L, K=8)
+    if mode == "topk_single_level":
+        return llsa.Problem(batch=batch, heads=heads, height=side, width=side, d=64, B=16, L=1, K=8)
+    return llsa.Problem(batch=batch, heads=heads, height=side, width=side, d=64, B=16, L=1, K=10 ** 6,
+                        enrich_mask=0)
+
+
+def run_sweep(args, local):
+    import torch
+
+    import synthetic
+    from hierarchical_top_sparse_b200 import llsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    out = []
+    for side in SWEEP_SIDES:
+        for mode in ("llsa", "topk_single_level", "dense"):
+            p = sweep_problem(llsa, side, mode)
+            n1 = p.N // p.B
+            rec = {"sweep": "tokens/s vs N", "N": p.N, "side": side, "mode": mode, "batch": p.batch,
+                   "heads": p.heads, "L": p.L, "K": min(p.K, n1), "enrich_mask": p.enrich_mask}
+            if mode == "dense" and n1 > DENSE_MAX_BLOCKS:
+                rec["skipped"] = (f"K_1 = {n1} blocks exceeds the tensor-core paths' {DENSE_MAX_BLOCKS}; "
+                                  "the index list alone would be " f"{p.batch * p.heads * n1 * n1 * 4 / 1e9:.1f} GB")
+                print(json.dumps(rec), flush=True)
+                out.append(rec)
+                continue
+            q, k, v = synthetic.qkv(side, p.batch, p.heads, side, side, p.d, 4.0 if side <= 256 else 8.0)
+            g = synthetic.upstream_grad(side + 1, p.batch, p.heads, p.N, p.d)
+            hier = []
+            for x in (q, k, v, g):
+                r = torch.from_numpy(x).to(dev).to(torch.bfloat16)
+                h = torch.empty_like(r)
+                llsa.reorder(p, r, h, True)
+                hier.append(h)
+                del r
+            qd, kd, vd, gd = hier
+            pipe = llsa.Pipeline(p, device=dev)
+
+            def sel():
+                llsa.pool(p, qd, pipe.pyrQ)
+                llsa.pool(p, kd, pipe.pyrK)
+                llsa.pool(p, vd, pipe.pyrV)
+                llsa.select(p, pipe.pyrQ, pipe.pyrK, pipe.idx)
+
+            def fwd():
+                llsa.attn_fwd(p, qd, kd, vd, pipe.pyrK, pipe.pyrV, pipe.idx, pipe.o, pipe.lse)
+
+            def bwd():
+                llsa.index_transpose(p, pipe.idx, pipe.offs, pipe.qlist, pipe.tscratch)
+                llsa.attn_bwd(p, qd, kd, vd, pipe.o, gd, pipe.lse, pipe.pyrK, pipe.pyrV, pipe.idx, pipe.offs,
+                              pipe.qlist, pipe.dq, pipe.dk, pipe.dv, pipe.work)
+
+            parts = (fwd, bwd) if mode == "dense" else (sel, fwd, bwd)
+            if mode == "dense":
+                sel()                      # the full index lists, once, untimed
+            steps = args.sweep_steps if mode != "dense" or side <= 128 else max(2, args.sweep_steps // 5)
+            for _ in range(2):
+                for f in parts:
+                    f()
+            torch.cuda.synchronize()
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)] for _ in range(steps)]
+            for i in range(steps):
+                evs[i][0].record(stream)
+                for j, f in enumerate(parts):
+                    f()
+                    evs[i][j + 1].record(stream)
+            torch.cuda.synchronize()
+            if llsa.device_error() != 0:
+                raise RuntimeError("a bounded device wait gave up during the sweep")
+            ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)) / steps
+                  for j in range(len(parts))]
+            names = ("attn_fwd", "transpose+attn_bwd") if mode == "dense" else ("pool+select", "attn_fwd",
+                                                                                 "transpose+attn_bwd")
+            tokens = p.batch * p.heads * p.N
+            rec.update({"steps": steps, "ms": {nm: round(t, 4) for nm, t in zip(names, ms)},
+                        "step_ms": round(sum(ms), 4),
+                        "fwd_tokens_per_s": round(tokens / ((sum(ms) - ms[-1]) / 1e3), 1),
+                        "bwd_tokens_per_s": round(tokens / (ms[-1] / 1e3), 1),
+                        "fwd_bwd_tokens_per_s": round(tokens / (sum(ms) / 1e3), 1),
+                        "attn_paths": llsa.attn_paths(p)})
+            print(json.dumps(rec), flush=True)
+            out.append(rec)
+            del pipe, qd, kd, vd, gd, hier
+            torch.cuda.empty_cache()
+    # speed-up of LLSA over dense at every N where both ran (forward: the
+    # inference figure; forward + backward: a training step's attention)
+    by = {(r["side"], r["mode"]): r for r in out}
+    for side in SWEEP_SIDES:
+        a, d = by.get((side, "llsa")), by.get((side, "dense"))
+        if a and d and "skipped" not in d:
+            print(json.dumps({"sweep": "speed-up vs dense", "side": side, "N": a["N"],
+                              "fwd": round(a["fwd_tokens_per_s"] / d["fwd_tokens_per_s"], 2),
+                              "fwd_bwd": round(a["fwd_bwd_tokens_per_s"] / d["fwd_bwd_tokens_per_s"], 2)}),
+                  flush=True)
+
+
 def llsa_pin(torch, t):
     h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
     h.copy_(t)
@@ -661,10 +779,17 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="px256",
                     help="the workload to time (default: the one the metric is quoted on)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the metric's line: tokens/s against N for LLSA, single-level top-K and "
+                         "dense attention, one JSON line per point (one GPU)")
+    ap.add_argument("--sweep-steps", type=int, default=10)
     args = ap.parse_args()
     select_workload(args.workload)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if args.sweep:
+        run_sweep(args, int(os.environ.get("LOCAL_RANK", "0")))
+        return
     rank, local, world, pg = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
