@@ -273,7 +273,11 @@ def traffic_record(kernel_stage: str):
 
 # The sources each stage's kernels are built from (the shared headers included).
 STAGE_SOURCES = {
+    "reorder": ("k_reorder_pool.cu",),
+    "pool": ("k_reorder_pool.cu",),
+    "select": ("k_select.cu",),
     "attn_fwd": ("k_attn_fwd_tc.cu",),
+    "index_transpose": ("k_transpose.cu",),
     "attn_bwd": ("k_attn_bwd.cu", "k_attn_bwd_q_tc.cu", "k_attn_bwd_kv_tc.cu"),
 }
 SHARED_HEADERS = ("llsa_internal.cuh", "ptx.cuh", "tcgen05.cuh")
@@ -565,7 +569,8 @@ def run_sweep(args, local):
         for mode in ("llsa", "topk_single_level", "dense"):
             p = sweep_problem(llsa, side, mode)
             n1 = p.N // p.B
-            rec = {"sweep": "tokens/s vs N", "N": p.N, "side": side, "mode": mode, "batch": p.batch,
+            rec = {"sweep": "tokens/s vs N", "tokens": "query rows (batch x heads x N)", "N": p.N, "side": side,
+                   "mode": mode, "batch": p.batch,
                    "heads": p.heads, "L": p.L, "K": min(p.K, n1), "enrich_mask": p.enrich_mask}
             if mode == "dense" and n1 > DENSE_MAX_BLOCKS:
                 rec["skipped"] = (f"K_1 = {n1} blocks exceeds the tensor-core paths' {DENSE_MAX_BLOCKS}; "
