@@ -33,7 +33,7 @@
 // rescales O (in TMEM) only when a new logit exceeds m by more than 2^8, so
 // the weights stay below 256 and O is rarely touched.
 //
-// Warp roles, one CTA per SM (24 warps):
+// Warp roles, one CTA per SM (25 warps):
 //   * warp 23, union: forms each group's union of picks -- with at most 64
 //     picks (K_1 <= 8, prefetched into registers a group ahead) by a
 //     warp-wide bitonic sort of (block, query block) keys, otherwise by
@@ -48,8 +48,9 @@
 //     three slots as the current group starts.  Issuing a TMA copy costs about
 //     a hundred cycles whatever its size, so the boxes follow runs and two
 //     warps issue in parallel;
-//   * warp 22, MMA: a converged warp whose elected lane issues every MMA, the
-//     S of entry i + 1 ahead of the O update of entry i;
+//   * warps 22 and 24, MMA: converged warps whose elected lanes issue every
+//     S (warp 22) and every O update (warp 24), so that the S of the next
+//     entries never queues behind the issue of an O update;
 //   * warps 0-15, softmax: one query row per thread; the four warps of a TMEM
 //     subpartition take two key blocks of a chunk each (pooled keys: 16 each
 //     in the first two), find their part of the row maximum and exchange it
@@ -83,16 +84,16 @@ constexpr int STAGE = 512;          // pick-list words a group stages in shared 
 constexpr int SOFT_WARPS = 16;      // four per TMEM subpartition, each on two of a chunk's key blocks
 constexpr int PARTS = SOFT_WARPS / 4;
 constexpr int NPROD = 2;            // producer warps, on alternate entries
-constexpr int EPI0 = 16, PRODUCER0 = 20, MMA_WARP = 22, UNION_WARP = 23;
-constexpr int THREADS = 24 * 32;
+constexpr int EPI0 = 16, PRODUCER0 = 20, MMA_WARP = 22, UNION_WARP = 23, PV_WARP = 24;
+constexpr int THREADS = 25 * 32;
 constexpr uint32_t TMEM_COLS = 512;
 // S of entry buffer b at 128 b, its P (bf16 pairs) at 256 + 64 b, O of group buffer o at 384 + 64 o
 constexpr uint32_t COL_S = 0, COL_P = 256, COL_O = 384;
 constexpr unsigned kNone = 0x7fffffffu;
 enum : int { kEnd = 0, kChunk = 1, kCoarse = 2, kGroupEnd = 3 };
 constexpr int kFirst = 1;           // first entry of a group
-// an entry is read by the MMA warp, every softmax warp and the producer that loads it
-constexpr int META_ARRIVALS = 1 + SOFT_WARPS + 1;
+// an entry is read by the two MMA warps, every softmax warp and the producer that loads it
+constexpr int META_ARRIVALS = 2 + SOFT_WARPS + 1;
 
 struct ChunkSlot {
   alignas(1024) unsigned char k[CK * 2048];    // [128 keys][64] bf16, 128-byte swizzle
@@ -135,7 +136,7 @@ struct Smem {
   uint64_t o_full[2], o_empty[2];              // O buffers: MMA -> epilogue, epilogue (4 warps) -> MMA / softmax
   uint64_t st_full[2];                         // row statistics: softmax warps -> epilogue
   uint64_t xbar[4];                            // the softmax warps of a subpartition exchange their maxima
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
 };
 
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       ptx::mbar_init(&s.st_full[i], SOFT_WARPS);
     }
     for (int i = 0; i < 4; ++i) ptx::mbar_init(&s.xbar[i], PARTS);
-    ptx::mbar_init(&s.drain, 1);
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(&s.drain[i], 1);
     ptx::fence_mbar_init();
   }
   // Rows of absent key blocks in a partial chunk keep whatever the slot held;
@@ -536,11 +537,15 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       }
     }
     __syncwarp();
-  } else if (warp == MMA_WARP) {
+  } else if (warp == MMA_WARP || warp == PV_WARP) {
     // ============================================================ MMA issue
-    // Converged warp, one elected lane issues.  Descriptors are built once and
-    // advanced by adding to their start-address field (16-byte units, no
-    // carry: shared addresses are below 256 KB).
+    // Two converged warps, one elected lane each: warp MMA_WARP issues every
+    // S, warp PV_WARP every O update, so that S of entry i + 1 never waits
+    // behind the issue of entry i's O update (which blocks while the tensor
+    // pipe works through S).  Each reads every entry; commits track only the
+    // issuing thread's MMAs.  Descriptors are built once and advanced by
+    // adding to their start-address field (16-byte units, no carry: shared
+    // addresses are below 256 KB).
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S: A = Q (K-major), B = K (K-major)
     constexpr uint32_t idSc = tc::idesc_bf16(128, 32, 0, 0);   // the same against the 32 pooled keys
     constexpr uint32_t idO = tc::idesc_bf16(128, 64, 0, 1);    // O += P V: A = P (TMEM), B = V (MN-major)
@@ -551,50 +556,53 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
     const uint64_t dv0 = tc::sw128_desc(ptx::smem_u32(s.slot[0].v), 16, 1024);
     const uint64_t dck0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].k), 16, 1024);
     const uint64_t dcv0 = tc::sw128_desc(ptx::smem_u32(s.crs[0].v), 16, 1024);
+    const bool is_s = warp == MMA_WARP;
     bool ok = true;
     uint32_t seen = 0, sidx = 0;
-    struct Entry { int kind, nq; uint32_t gc, tk, kc, sb; int msk[CK]; };
+    bool o_started = false;   // O update warp: the group has taken its O buffer
     auto wait = [&](uint64_t* bar, uint32_t parity) {
       if (ok && !ptx::mbar_wait_bounded(bar, parity, kWaitLimitNs)) ok = false;
       return ok;
     };
-    // Reads the next entry and issues its S; false on the end marker or a timeout.
-    auto next_s = [&](Entry& c) -> bool {
+    while (ok) {
       const int ms = (int)(seen % NMETA);
-      if (!wait(&s.mfull[ms], (seen / NMETA) & 1)) return false;
+      if (!wait(&s.mfull[ms], (seen / NMETA) & 1)) break;
       const Meta& m = s.meta[ms];
-      c.kind = m.kind;
-      c.nq = m.nq;
-      c.gc = (uint32_t)m.gc;
-      c.tk = (uint32_t)m.tk;
-      c.kc = (uint32_t)m.kc;
+      const int kind = m.kind, nq = m.nq, flags = m.flags;
+      const uint32_t gc = (uint32_t)m.gc, tk = (uint32_t)m.tk, kc = (uint32_t)m.kc;
+      int msk[CK];
 #pragma unroll
-      for (int j = 0; j < CK; ++j) c.msk[j] = m.msk[j];
-      const int flags = m.flags;
+      for (int j = 0; j < CK; ++j) msk[j] = m.msk[j];
       __syncwarp();
       if (tc::elect_one()) ptx::mbar_arrive(&s.mempty[ms]);   // the entry is in registers
       __syncwarp();
       ++seen;
-      if (c.kind == kEnd) return false;
-      const uint32_t qs = c.gc % NQ;
-      if ((flags & kFirst) && !wait(&s.qfull[qs], (c.gc / NQ) & 1)) return false;   // the group's Q has landed
-      const bool chunk = c.kind == kChunk && c.nq > 0;
-      const bool has_s = c.kind == kCoarse || chunk;
-      if (c.kind == kCoarse && (c.gc & 1) == 0 && !wait(&s.cfull[c.tk & 1], (c.tk >> 1) & 1)) return false;
-      if (chunk && !wait(&s.kfull[c.kc % NSLOT], (c.kc / NSLOT) & 1)) return false;
-      if (has_s) {
+      if (kind == kEnd) break;
+      const bool chunk = kind == kChunk && nq > 0;
+      const bool has_s = kind == kCoarse || chunk;
+      const uint32_t qs = gc % NQ, ob = gc & 1;
+      if (is_s) {
+        if (kind == kGroupEnd) {   // every S of the group has been issued: its Q is free once they finish
+          if (tc::elect_one()) tc::commit(&s.qempty[qs]);
+          __syncwarp();
+          continue;
+        }
+        if ((flags & kFirst) && !wait(&s.qfull[qs], (gc / NQ) & 1)) break;   // the group's Q has landed
+        if (kind == kCoarse && (gc & 1) == 0 && !wait(&s.cfull[tk & 1], (tk >> 1) & 1)) break;
+        if (chunk && !wait(&s.kfull[kc % NSLOT], (kc / NSLOT) & 1)) break;
+        if (!has_s) continue;
         const uint32_t b = sidx & 1, u = sidx >> 1;
-        if (!wait(&s.s_empty[b], (u & 1) ^ 1)) return false;   // the softmax warps have read S(b) of entry sidx - 2
+        if (!wait(&s.s_empty[b], (u & 1) ^ 1)) break;   // the softmax warps have read S(b) of entry sidx - 2
         tc::fence_after_sync();
         const uint64_t go = kQStep * (uint64_t)qs;
         if (tc::elect_one()) {
           if (chunk) {
-            const uint64_t so = kSlotStep * (uint64_t)(c.kc % NSLOT);
+            const uint64_t so = kSlotStep * (uint64_t)(kc % NSLOT);
 #pragma unroll
             for (int k = 0; k < 4; ++k)   // K steps of 16 channels: 32 bytes inside the 128-byte rows
               tc::mma_bf16(tbase + COL_S + 128u * b, dq0 + go + 2u * k, dk0 + so + 2u * k, idS, k > 0);
           } else {
-            const uint64_t co = kCrsStep * (uint64_t)(c.tk & 1);
+            const uint64_t co = kCrsStep * (uint64_t)(tk & 1);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               tc::mma_bf16(tbase + COL_S + 128u * b, dq0 + go + 2u * k, dck0 + co + 2u * k, idSc, k > 0);
@@ -602,76 +610,52 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
           tc::commit(&s.s_full[b]);
         }
         __syncwarp();
-        c.sb = sidx++;
-      }
-      return true;
-    };
-
-    // O of each group buffer starts at zero (the epilogue clears it after
-    // reading it), so every O update accumulates.
-    bool o_started = false;
-    auto finish = [&](const Entry& c) {
-      const uint32_t ob = c.gc & 1;
-      const bool chunk = c.kind == kChunk && c.nq > 0;
-      if (c.kind == kCoarse || chunk) {
-        const uint32_t b = c.sb & 1, u = c.sb >> 1;
-        if (!wait(&s.p_full[b], u & 1)) return;
-        // the group's first O update: its last group's epilogue has read and cleared the buffer
-        if (!o_started && !wait(&s.o_empty[ob], ((c.gc >> 1) & 1) ^ 1)) return;
-        tc::fence_after_sync();
-        const uint32_t oc = tbase + COL_O + 64u * ob, pc = tbase + COL_P + 64u * b;
-        if (tc::elect_one()) {
-          if (chunk) {
-            const uint64_t so = kSlotStep * (uint64_t)(c.kc % NSLOT);
+        ++sidx;
+      } else {
+        if (has_s) {
+          const uint32_t b = sidx & 1, u = sidx >> 1;
+          if (!wait(&s.p_full[b], u & 1)) break;
+          // the group's first O update: its last group's epilogue has read and cleared the buffer
+          if (!o_started && !wait(&s.o_empty[ob], ((gc >> 1) & 1) ^ 1)) break;
+          // V landed with K (the S warp saw it; the phase cannot have moved on
+          // before this warp frees the slot)
+          if (chunk && !wait(&s.kfull[kc % NSLOT], (kc / NSLOT) & 1)) break;
+          tc::fence_after_sync();
+          const uint32_t oc = tbase + COL_O + 64u * ob, pc = tbase + COL_P + 64u * b;
+          if (tc::elect_one()) {
+            if (chunk) {
+              const uint64_t so = kSlotStep * (uint64_t)(kc % NSLOT);
 #pragma unroll
-            for (int k = 0; k < CK; ++k) {   // key block k: A 8 TMEM columns, B 2 KB
-              if (k >= c.nq) break;
-              // rows of the query blocks that did not pick block k keep their O
-              const unsigned skip = ~(unsigned)c.msk[k] & 0xffu;
-              uint32_t off[4];
+              for (int k = 0; k < CK; ++k) {   // key block k: A 8 TMEM columns, B 2 KB
+                if (k >= nq) break;
+                tc::mma_bf16_ta(oc, pc + 8u * k, dv0 + so + 128u * k, idO, true);
+              }
+              tc::commit(&s.kempty[kc % NSLOT]);
+            } else {
+              const uint64_t co = kCrsStep * (uint64_t)(tk & 1);
 #pragma unroll
-              for (int w = 0; w < 4; ++w)
-                off[w] = (((skip >> (2 * w)) & 1u) ? 0x0000ffffu : 0u) | (((skip >> (2 * w + 1)) & 1u) ? 0xffff0000u : 0u);
-              tc::mma_bf16_ta_rows(oc, pc + 8u * k, dv0 + so + 128u * k, idO, true, off[0], off[1], off[2], off[3]);
+              for (int k = 0; k < 2; ++k) tc::mma_bf16_ta(oc, pc + 8u * k, dcv0 + co + 128u * k, idO, true);
+              if (gc & 1) tc::commit(&s.cempty[tk & 1]);
             }
-            tc::commit(&s.kempty[c.kc % NSLOT]);
-          } else {
-            const uint64_t co = kCrsStep * (uint64_t)(c.tk & 1);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) tc::mma_bf16_ta(oc, pc + 8u * k, dcv0 + co + 128u * k, idO, true);
-            if (c.gc & 1) tc::commit(&s.cempty[c.tk & 1]);
+            tc::commit(&s.p_empty[b]);
           }
-          tc::commit(&s.p_empty[b]);
+          __syncwarp();
+          o_started = true;
+          ++sidx;
+        } else if (kind == kGroupEnd) {
+          // no O update in this group: still take the buffer over in order
+          if (!o_started && !wait(&s.o_empty[ob], ((gc >> 1) & 1) ^ 1)) break;
+          if (tc::elect_one()) tc::commit(&s.o_full[ob]);   // the group's O is complete
+          __syncwarp();
+          o_started = false;
         }
-        __syncwarp();
-        o_started = true;
-      } else if (c.kind == kGroupEnd) {
-        // no O update in this group: still take the buffer over in order
-        if (!o_started && !wait(&s.o_empty[ob], ((c.gc >> 1) & 1) ^ 1)) return;
-        if (tc::elect_one()) {
-          tc::commit(&s.o_full[ob]);              // the group's O is complete
-          tc::commit(&s.qempty[c.gc % NQ]);       // its Q is free
-        }
-        __syncwarp();
-        o_started = false;
       }
-    };
-
-    Entry cur;
-    bool have = next_s(cur);
-    while (have && ok) {
-      Entry nxt;
-      const bool have_next = next_s(nxt);
-      if (!ok) break;
-      finish(cur);
-      cur = nxt;
-      have = have_next;
     }
-    if (!ok && lane == 0) report(err, 77);
+    if (!ok && lane == 0) report(err, is_s ? 77 : 76);
     // every MMA issued here has finished before TMEM is released
-    if (tc::elect_one()) tc::commit(&s.drain);
+    if (tc::elect_one()) tc::commit(&s.drain[is_s ? 0 : 1]);
     __syncwarp();
-    ptx::mbar_wait_bounded(&s.drain, 0, kWaitLimitNs);
+    ptx::mbar_wait_bounded(&s.drain[is_s ? 0 : 1], 0, kWaitLimitNs);
   } else if (warp < SOFT_WARPS) {
     // ============================================================ softmax
     // The four warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4)..
@@ -803,11 +787,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       // the O update skips the rows that did not pick a block
 #pragma unroll 1
       for (int jj = 0; jj < nblk; ++jj) {
-        if (!((need >> jj) & 1u)) continue;
+        uint32_t pw[8];
+        if (!((need >> jj) & 1u)) {
+#pragma unroll
+          for (int n = 0; n < 8; ++n) pw[n] = 0u;
+          tc::tmem_st8(tl + pcol0 + 8u * jj, pw);
+          continue;
+        }
         uint32_t sr[16];
         tc::tmem_ld16(tl + scol0 + 16u * jj, sr);
         tc::tmem_wait_ld();
-        uint32_t pw[8];
         if ((mine >> jj) & 1u) {
           float sh = 0.f;
           if (!coarse && enrich1) {
