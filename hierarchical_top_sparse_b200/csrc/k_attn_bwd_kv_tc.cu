@@ -67,8 +67,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int CQ = 8;               // query blocks per chunk (128 queries)
 constexpr int KG = 8;               // key blocks per group (128 keys)
 constexpr int NSLOT = 3;            // chunk slots
-constexpr int SOFT_WARPS = 16, PRODUCER_WARP = 20, MMA_WARP = 21;   // warps 16-19: epilogue
-constexpr int THREADS = 22 * 32;
+constexpr int SOFT_WARPS = 16, PRODUCER_WARP = 20, MMA_WARP = 21, GRAD_WARP = 22;   // warps 16-19: epilogue
+constexpr int THREADS = 23 * 32;
 constexpr uint32_t TMEM_COLS = 512;
 // S 0-127, dP 128-255; accumulator buffer b at 256 + 128 b: dV + 0, dK + 64
 constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
@@ -109,7 +109,7 @@ struct Smem {
   uint64_t p_full, p_empty;                    // P / dS operands: softmax (8 warps) -> MMA, MMA -> softmax
   uint64_t acc_full[2], acc_empty[2];          // accumulator buffers: MMA -> epilogue, epilogue (4 warps) -> MMA
   uint64_t gid_full[GRING], gid_empty[GRING];  // the CTA's key groups in claim order: producer -> epilogue
-  uint64_t drain;
+  uint64_t drain[2];
   int gid[GRING];
   uint32_t tmem_base;
 };
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       ptx::mbar_init(&s.gid_full[i], 1);
       ptx::mbar_init(&s.gid_empty[i], 4);
     }
-    ptx::mbar_init(&s.drain, 1);
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(&s.drain[i], 1);
     ptx::fence_mbar_init();
   }
   // Rows of absent query blocks in a partial chunk keep whatever the slot
@@ -340,14 +340,18 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
         ptx::mbar_wait_bounded(&s.kfull[i & 1], (i >> 1) & 1, kWaitLimitNs);
     }
     __syncwarp();
-  } else if (warp == MMA_WARP) {
+  } else if (warp == MMA_WARP || warp == GRAD_WARP) {
     // ============================================================ MMA issue
-    // Converged warp, one elected lane issues.  Descriptors are built once and
-    // advanced by adding to their start-address field (16-byte units, no
-    // carry: shared addresses are below 256 KB).  Software-pipelined: S and
-    // dP of chunk i + 1 are issued as soon as the softmax warps have read
-    // those of chunk i, before dV / dK of chunk i, so that the tensor cores
-    // work while the softmax warps do.
+    // Two converged warps, one elected lane each: warp MMA_WARP issues S and
+    // dP of every chunk (as soon as the softmax warps have read those of the
+    // chunk before), warp GRAD_WARP dV and dK (once the softmax warps have
+    // written P and dS), so that neither issue stream waits behind the other.
+    // Each reads every chunk's meta words; commits track only the issuing
+    // thread's MMAs (S and dP of a chunk have finished before its P / dS
+    // exist, so GRAD_WARP's commits cover the chunk and the group).
+    // Descriptors are built once and advanced by adding to their
+    // start-address field (16-byte units, no carry: shared addresses are
+    // below 256 KB).
     constexpr uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);   // S, dP: A = Q / dO (K-major), B = K / V (K-major)
     constexpr uint32_t idG = tc::idesc_bf16(128, 64, 1, 1);    // dV, dK: A = P / dS (MN-major), B = dO / Q (MN-major)
     constexpr uint64_t kSlotStep = sizeof(ChunkSlot) >> 4, kKeyStep = sizeof(KeySlot) >> 4;
@@ -357,42 +361,31 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
     const uint64_t dv0 = tc::sw128_desc(ptx::smem_u32(s.key[0].v), 16, 1024);
     const uint64_t dp = tc::sw128_desc(ptx::smem_u32(s.pbuf), 16384, 1024);
     const uint64_t dsd = tc::sw128_desc(ptx::smem_u32(s.sbuf), 16384, 1024);
+    const bool is_s = warp == MMA_WARP;
     bool ok = true;
-    uint32_t seen = 0;        // chunks whose meta words were read (the S side runs one chunk ahead)
-    uint32_t sch = 0;         // chunks with queries whose S / dP were issued
-    uint32_t kseen = 0;       // groups started on the S side
-    // Reads the next chunk's meta and, if it has queries, issues its S / dP.
-    // Returns false on the end marker or a timeout.
-    struct Chunk { int slot, nq, flags, ks; };
-    auto next_s = [&](Chunk& c) -> bool {
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+      if (ok && !ptx::mbar_wait_bounded(bar, parity, kWaitLimitNs)) ok = false;
+      return ok;
+    };
+    uint32_t kseen = 0;           // groups started
+    uint32_t nch = 0;             // chunks with queries handled
+    uint32_t gcount = 0;          // groups closed (GRAD_WARP)
+    bool in_group = false;
+    for (uint32_t seen = 0; ok; ++seen) {
       const int slot = (int)(seen % NSLOT);
-      if (!ptx::mbar_wait_bounded(&s.full[slot], (seen / NSLOT) & 1, kWaitLimitNs)) {
-        ok = false;
-        return false;
-      }
+      if (!wait(&s.full[slot], (seen / NSLOT) & 1)) break;
       const Meta& m = s.meta[slot];
-      if (m.kind == kEnd) return false;
-      c.slot = slot;
-      c.nq = m.nq;
-      c.flags = m.flags;
-      if (c.flags & kFirst) {
-        const int ks = (int)(kseen & 1);
-        if (!ptx::mbar_wait_bounded(&s.kfull[ks], (kseen >> 1) & 1, kWaitLimitNs)) {
-          ok = false;
-          return false;
-        }
-        ++kseen;
-      }
-      c.ks = (int)((kseen - 1) & 1);
-      ++seen;
-      if (c.nq > 0) {
+      const int kind = m.kind, nq = m.nq, flags = m.flags;
+      if (kind == kEnd) break;
+      if (flags & kFirst) ++kseen;
+      const int ks = (int)((kseen - 1) & 1);
+      if (is_s) {
+        if ((flags & kFirst) && !wait(&s.kfull[ks], ((kseen - 1) >> 1) & 1)) break;
+        if (nq == 0) continue;
         // the softmax warps have read S / dP of the previous chunk
-        if (!ptx::mbar_wait_bounded(&s.s_empty, (sch & 1) ^ 1, kWaitLimitNs)) {
-          ok = false;
-          return false;
-        }
+        if (!wait(&s.s_empty, (nch & 1) ^ 1)) break;
         tc::fence_after_sync();
-        const uint64_t so = kSlotStep * (uint64_t)slot, ko = kKeyStep * (uint64_t)c.ks;
+        const uint64_t so = kSlotStep * (uint64_t)slot, ko = kKeyStep * (uint64_t)ks;
         if (tc::elect_one()) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {   // K steps of 16 channels: 32 bytes inside the 128-byte rows
@@ -402,34 +395,17 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
           tc::commit(&s.s_full);
         }
         __syncwarp();
-        ++sch;
+        ++nch;
+        continue;
       }
-      return true;
-    };
-
-    uint32_t pch = 0, gcount = 0;   // chunks with queries whose dV / dK were issued; groups closed
-    bool in_group = false;
-    Chunk cur;
-    bool have = next_s(cur);
-    while (have && ok) {
-      Chunk nxt;
-      const bool have_next = next_s(nxt);
-      if (!ok) break;
-      // dV / dK of the current chunk
-      if (cur.nq > 0) {
-        if (!ptx::mbar_wait_bounded(&s.p_full, pch & 1, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+      // dV / dK of this chunk
+      if (nq > 0) {
+        if (!wait(&s.p_full, nch & 1)) break;
         const uint32_t b = gcount & 1;
-        if (!in_group) {   // the group's first MMA overwrites the buffer: wait until it was read
-          if (!ptx::mbar_wait_bounded(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-        }
+        // the group's first MMA overwrites the buffer: wait until it was read
+        if (!in_group && !wait(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1)) break;
         tc::fence_after_sync();
-        const uint64_t so = kSlotStep * (uint64_t)cur.slot;
+        const uint64_t so = kSlotStep * (uint64_t)slot;
         const uint32_t acc = tbase + COL_ACC + 128u * b;
         if (tc::elect_one()) {
 #pragma unroll
@@ -438,39 +414,33 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
             tc::mma_bf16(acc + 64, dsd + 128u * k, dq0 + so + 128u * k, idG, in_group || k > 0);
           }
           tc::commit(&s.p_empty);
-          tc::commit(&s.empty[cur.slot]);
+          tc::commit(&s.empty[slot]);
         }
         __syncwarp();
         in_group = true;
-        ++pch;
+        ++nch;
       } else {
-        if (tc::elect_one()) ptx::mbar_arrive(&s.empty[cur.slot]);
+        if (tc::elect_one()) ptx::mbar_arrive(&s.empty[slot]);
         __syncwarp();
       }
-      if (cur.flags & kLast) {
+      if (flags & kLast) {
         const uint32_t b = gcount & 1;
-        if (!in_group) {   // no MMA in this group: still hand the buffer over in order
-          if (!ptx::mbar_wait_bounded(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-        }
+        // no MMA in this group: still hand the buffer over in order
+        if (!in_group && !wait(&s.acc_empty[b], ((gcount >> 1) & 1) ^ 1)) break;
         if (tc::elect_one()) {
-          tc::commit(&s.kempty[cur.ks]);   // the group's K and V are free once its MMAs are done
+          tc::commit(&s.kempty[ks]);   // the group's K and V are free once its MMAs are done
           tc::commit(&s.acc_full[b]);
         }
         __syncwarp();
         ++gcount;
         in_group = false;
       }
-      cur = nxt;
-      have = have_next;
     }
-    if (!ok && lane == 0) report(err, 44);
+    if (!ok && lane == 0) report(err, is_s ? 44 : 49);
     // every MMA issued here has finished before TMEM is released
-    if (tc::elect_one()) tc::commit(&s.drain);
+    if (tc::elect_one()) tc::commit(&s.drain[is_s ? 0 : 1]);
     __syncwarp();
-    ptx::mbar_wait_bounded(&s.drain, 0, kWaitLimitNs);
+    ptx::mbar_wait_bounded(&s.drain[is_s ? 0 : 1], 0, kWaitLimitNs);
   } else if (warp < SOFT_WARPS) {
     // ============================================================ softmax
     const int sub = warp & 3, part = warp >> 2;         // TMEM subpartition; key blocks 2 part, 2 part + 1

@@ -651,7 +651,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
         }
       }
     }
-    if (!ok && lane == 0) report(err, is_s ? 77 : 76);
+    if (!ok && lane == 0) report(err, is_s ? 77 : 75);
     // every MMA issued here has finished before TMEM is released
     if (tc::elect_one()) tc::commit(&s.drain[is_s ? 0 : 1]);
     __syncwarp();
