@@ -10,6 +10,7 @@
 // the list, and a ballot pass writes it out in ascending key order (candidate
 // ids grow with the candidate position because parent lists are ascending).
 #include "llsa_internal.cuh"
+#include "ptx.cuh"
 
 namespace llsa {
 
@@ -99,148 +100,182 @@ __global__ void select_level_kernel(Geo g, int l, const float* __restrict__ pyrQ
   }
 }
 
-// ------------------------------------------------ child search, one CTA per parent
+// ------------------------------------------------ child search, pipelined over parents
 //
-// The B sibling query tokens under one level-(l+1) token share their
-// candidates (the B children of each of the parent's picks), so one CTA
-// loads those candidate rows once into shared memory and scores the whole
-// B x (K_{l+1} B) tile: every thread a 4 x 4 register tile of scores, each a
-// sequential fp32 FMA chain over d (the same rounding as the one-warp kernel
-// above).  Then one warp per query token takes K_l rounds of a warp-wide max
-// over 64-bit keys held in registers and writes the picks in ascending order.
+// The B sibling query tokens under one level-(l+1) token (a parent) share
+// their candidates: the B children of each of the parent's picks.  A CTA
+// walks parents in grid-stride order with two shared-memory stages: the
+// candidate rows and the 16 query rows of parent i + 2 are copied in
+// (16-byte asynchronous copies into padded rows) while the CTA scores parent
+// i.  Every thread scores a 2 x 4 register tile (2 query rows of its warp x
+// candidates lane + 32 j), each a sequential fp32 FMA chain over the 64
+// channels; then the warp takes K_l rounds of a warp-wide maximum for each of
+// its rows (two one-instruction reductions per round: the orderable score,
+// then, among the lanes that hold it, the lower candidate position) and
+// writes the picks in ascending order.
 namespace selchild {
-constexpr int THREADS = 128;
-constexpr int NC = 128;        // candidates per parent, at most
+constexpr int THREADS = 256;
+constexpr int NC = 128;        // candidates per parent, at most (K_{l+1} <= 8)
 constexpr int QB = 16;         // sibling query tokens (B)
 constexpr int LD = 68;         // padded row length (floats): conflict-free 16-byte reads
+constexpr int STAGES = 2;
+struct Stage {
+  float k[NC * LD];            // candidate m = child m % B of pick m / B
+  float q[QB * LD];            // the parent's 16 query rows
+};
+constexpr size_t kSmem = sizeof(Stage) * STAGES;
 }
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __global__ void __launch_bounds__(selchild::THREADS) select_children_kernel(Geo g, int l,
                                                                             const float* __restrict__ pyrQ,
                                                                             const float* __restrict__ pyrK,
                                                                             int32_t* __restrict__ idx) {
   using namespace selchild;
-  __shared__ __align__(16) float ks[NC * LD];
-  __shared__ __align__(16) float qs[QB * LD];
-  __shared__ int cid[NC];
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  Stage* st = reinterpret_cast<Stage*>(sm_raw);
+  __shared__ int cids[STAGES][NC];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nl = g.n[l], np = g.n[l + 1];
-  const int bh = blockIdx.x / np;
-  const int par = blockIdx.x - bh * np;
   const int Kp = g.Kl[l + 1], Kl = g.Kl[l];
   const int ncand = Kp * QB;
-  const int32_t* plist = idx + g.idx_off[l + 1] + ((int64_t)bh * np + par) * Kp;
-  const float* kbase = pyrK + g.pyr_off[l] + (int64_t)bh * nl * 64;
-  const float* qbase = pyrQ + g.pyr_off[l] + ((int64_t)bh * nl + (int64_t)par * QB) * 64;
+  const int64_t nparents = (int64_t)g.BH * np;
+  const int64_t stride = gridDim.x;
 
-  // Candidate m is child m % B of pick m / B.  Every thread resolves the ids of
-  // the rows it copies itself (the parent list is a few cached words), so the
-  // candidate rows and the query rows are fetched in one round.
-  auto cand = [&](int m) -> int {
-    if (m >= ncand) return -1;
-    const int pc = plist[m / QB];
-    return (pc >= 0 && pc < np) ? pc * QB + m % QB : -1 - (pc * QB + m % QB);   // < 0: parent corrupted
+  // Stage sidx <- parent p (every thread copies its share); one copy group
+  // per call, empty when p is past the end.  Candidate ids < 0: the pick lies
+  // outside its level (-1 - the id the list implies), the candidate never wins.
+  auto issue = [&](int64_t p, int sidx) {
+    if (p < nparents) {
+      const int bh = (int)(p / np), par = (int)(p - (int64_t)bh * np);
+      const int32_t* plist = idx + g.idx_off[l + 1] + ((int64_t)bh * np + par) * Kp;
+      const float* kbase = pyrK + g.pyr_off[l] + (int64_t)bh * nl * 64;
+      const float* qbase = pyrQ + g.pyr_off[l] + ((int64_t)bh * nl + (int64_t)par * QB) * 64;
+      if (tid < NC) {
+        int c = -1;
+        if (tid < ncand) {
+          const int pc = plist[tid / QB];
+          c = (pc >= 0 && pc < np) ? pc * QB + tid % QB : -1 - (pc * QB + tid % QB);
+        }
+        cids[sidx][tid] = c;
+      }
+      for (int e = tid; e < (NC + QB) * 16; e += THREADS) {
+        const int r = e >> 4, c4 = (e & 15) * 4;
+        if (r < NC) {
+          if (r < ncand) {
+            const int pc = plist[r / QB];
+            if (pc >= 0 && pc < np) cp_async16(&st[sidx].k[r * LD + c4], kbase + ((int64_t)pc * QB + r % QB) * 64 + c4);
+          }
+        } else {
+          cp_async16(&st[sidx].q[(r - NC) * LD + c4], qbase + (r - NC) * 64 + c4);
+        }
+      }
+    }
+    cp_async_commit();
   };
-  if (tid < NC) cid[tid] = cand(tid);
-  for (int e = tid; e < QB * 16; e += THREADS) {
-    const int r = e >> 4, c4 = (e & 15) * 4;
-    *reinterpret_cast<float4*>(&qs[r * LD + c4]) = *reinterpret_cast<const float4*>(qbase + r * 64 + c4);
-  }
-  for (int e = tid; e < NC * 16; e += THREADS) {
-    const int m = e >> 4, c4 = (e & 15) * 4;
-    const int c = cand(m);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (c >= 0) v = *reinterpret_cast<const float4*>(kbase + (int64_t)c * 64 + c4);
-    *reinterpret_cast<float4*>(&ks[m * LD + c4]) = v;
-  }
-  __syncthreads();
 
-  // scores: warp w takes query rows 4w..4w+3, lane the candidates lane + 32 j;
-  // they stay in registers
-  float acc[4][4];
+  const int64_t first = blockIdx.x;
+  issue(first, 0);
+  issue(first + stride, 1);
+  uint32_t it = 0;
+  for (int64_t p = first; p < nparents; p += stride, ++it) {
+    const int sidx = (int)(it & 1);
+    cp_async_wait_one();   // this stage's copies (the next stage's may still fly)
+    __syncthreads();
+    const Stage& S = st[sidx];
+    // scores: warp w takes query rows 2w, 2w+1, lane the candidates lane + 32 j
+    float acc[2][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int e = 0; e < 64; e += 4) {
-    float4 qv[4], kv[4];
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int e = 0; e < 64; e += 4) {
+      float4 qv[2], kv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const float4*>(&qs[(warp * 4 + i) * LD + e]);
+      for (int i = 0; i < 2; ++i) qv[i] = *reinterpret_cast<const float4*>(&S.q[(warp * 2 + i) * LD + e]);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) kv[j] = *reinterpret_cast<const float4*>(&ks[(lane + 32 * j) * LD + e]);
+      for (int j = 0; j < 4; ++j) kv[j] = *reinterpret_cast<const float4*>(&S.k[(lane + 32 * j) * LD + e]);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
-        acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
-        acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
-        acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
-      }
-  }
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
+        }
+    }
+    int cid[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cid[j] = cids[sidx][lane + 32 * j];
+    const int bh = (int)(p / np), par = (int)(p - (int64_t)bh * np);
+    __syncthreads();   // every read of this stage is done: refill it
+    issue(p + 2 * stride, sidx);
 
-  // top-K_l of the warp's 4 rows, the 4 rows' rounds interleaved so that their
-  // shuffle chains overlap: 64-bit keys (orderable score, then the lower
-  // candidate position wins a tie)
-  uint64_t key[4][4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int m = lane + 32 * j;
-    const int c = m < ncand ? cid[m] : 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (m >= ncand)
-        key[i][j] = 0;
-      else if (c < 0)
-        key[i][j] = 1ull << 32;          // parent corrupted: the candidate never wins
-      else
-        key[i][j] = ((uint64_t)orderable(acc[i][j]) << 32) | (uint64_t)(0xffffffffu - (uint32_t)m);
-    }
-  }
-  unsigned taken[4] = {0u, 0u, 0u, 0u};
-  for (int k = 0; k < Kl; ++k) {
-    uint64_t best[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      best[i] = key[i][0];
-#pragma unroll
-      for (int j = 1; j < 4; ++j) best[i] = key[i][j] > best[i] ? key[i][j] : best[i];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint64_t w = __shfl_xor_sync(0xffffffffu, best[i], o);
-        best[i] = w > best[i] ? w : best[i];
-      }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = (int)(0xffffffffu - (uint32_t)best[i]);
-      const bool mine = (m & 31) == lane;
-      const int jj = m >> 5;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (mine && j == jj) key[i][j] = 0;
-      if (mine) taken[i] |= 1u << jj;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = warp * 4 + i;
-    int32_t* out = idx + g.idx_off[l] + ((int64_t)bh * nl + (int64_t)par * QB + r) * Kl;
-    int written = 0;
+    // keys: hi = orderable score (0: no score), lo = 128 - candidate position
+    // (0: no candidate or taken); the maximum (hi, lo) is the highest score,
+    // then the lowest position, i.e. the lowest key id
+    uint32_t hi[2][4], lo[2][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const bool t = (taken[i] >> j) & 1u;
-      const unsigned bal = __ballot_sync(0xffffffffu, t);
-      if (t) {
-        const int m = lane + 32 * j;
-        const int c = cid[m];
-        out[written + __popc(bal & ((1u << lane) - 1u))] = c >= 0 ? c : -1 - c;
+      const int m = lane + 32 * j;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (m >= ncand) {
+          hi[i][j] = 0u;
+          lo[i][j] = 0u;
+        } else {
+          hi[i][j] = cid[j] < 0 ? 0u : orderable(acc[i][j]);   // a pick outside its level: after every score
+          lo[i][j] = 128u - (uint32_t)m;
+        }
       }
-      written += __popc(bal);
+    }
+    unsigned taken[2] = {0u, 0u};
+    for (int k = 0; k < Kl; ++k) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        uint32_t bh_ = hi[i][0], bl_ = lo[i][0];
+#pragma unroll
+        for (int j = 1; j < 4; ++j)
+          if (hi[i][j] > bh_ || (hi[i][j] == bh_ && lo[i][j] > bl_)) {
+            bh_ = hi[i][j];
+            bl_ = lo[i][j];
+          }
+        const uint32_t H = __reduce_max_sync(0xffffffffu, bh_);
+        const uint32_t Lw = __reduce_max_sync(0xffffffffu, bh_ == H ? bl_ : 0u);
+        const int m = 128 - (int)Lw;
+        const bool mine = (m & 31) == lane;
+        const int jj = m >> 5;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (mine && j == jj) {
+            hi[i][j] = 0u;
+            lo[i][j] = 0u;
+          }
+        if (mine) taken[i] |= 1u << jj;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int r = warp * 2 + i;
+      int32_t* out = idx + g.idx_off[l] + ((int64_t)bh * nl + (int64_t)par * QB + r) * Kl;
+      int written = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool t = (taken[i] >> j) & 1u;
+        const unsigned bal = __ballot_sync(0xffffffffu, t);
+        if (t) out[written + __popc(bal & ((1u << lane) - 1u))] = cid[j] >= 0 ? cid[j] : -1 - cid[j];
+        written += __popc(bal);
+      }
     }
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight when the CTA leaves
 }
 
 cudaError_t launch_select_level(const Geo& g, int level, const float* pyrQ, const float* pyrK, int32_t* idx,
@@ -248,7 +283,15 @@ cudaError_t launch_select_level(const Geo& g, int level, const float* pyrQ, cons
   if (level < g.L && g.d == 64 && g.B == selchild::QB && g.Kl[level + 1] * g.B <= selchild::NC &&
       g.Kl[level] < g.Kl[level + 1] * g.B) {
     const int64_t parents = (int64_t)g.BH * g.n[level + 1];
-    select_children_kernel<<<(unsigned)parents, selchild::THREADS, 0, s>>>(g, level, pyrQ, pyrK, idx);
+    cudaError_t e = cudaFuncSetAttribute(select_children_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)selchild::kSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t resident = 2ll * sms;   // two CTAs of 77 KB per SM
+    const unsigned grid = (unsigned)(parents < resident ? parents : resident);
+    select_children_kernel<<<grid, selchild::THREADS, selchild::kSmem, s>>>(g, level, pyrQ, pyrK, idx);
     note_launches(1);
     return cudaGetLastError();
   }
