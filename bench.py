@@ -713,7 +713,7 @@ def oracle_setup():
     BH = w["batch"] * w["heads"]
     cores, _ = host_cpu()
     slices = min(BH, cores)
-    groups = max(1, cores // slices)
+    groups = max(1, -(-cores // slices))   # at least one thread per host core
     inputs = [oracle.reorder(op, x.reshape(BH, op.N, w["d"])[:slices], True) for x in (q, k, v, g)]
     return op, inputs, slices, groups
 

@@ -124,6 +124,7 @@ struct Stage {
   float q[QB * LD];            // the parent's 16 query rows
 };
 constexpr size_t kSmem = sizeof(Stage) * STAGES;
+static_assert((NC + QB) * 16 % THREADS == 0, "every thread copies the same number of 16-byte pieces");
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -156,21 +157,20 @@ __global__ void __launch_bounds__(selchild::THREADS) select_children_kernel(Geo 
       const int32_t* plist = idx + g.idx_off[l + 1] + ((int64_t)bh * np + par) * Kp;
       const float* kbase = pyrK + g.pyr_off[l] + (int64_t)bh * nl * 64;
       const float* qbase = pyrQ + g.pyr_off[l] + ((int64_t)bh * nl + (int64_t)par * QB) * 64;
+      // lane j of every warp holds pick j: one round of loads, then shuffles
+      const int pl = lane < Kp ? plist[lane] : -1;
       if (tid < NC) {
-        int c = -1;
-        if (tid < ncand) {
-          const int pc = plist[tid / QB];
-          c = (pc >= 0 && pc < np) ? pc * QB + tid % QB : -1 - (pc * QB + tid % QB);
-        }
-        cids[sidx][tid] = c;
+        const int pc = __shfl_sync(0xffffffffu, pl, (tid / QB) & 31);
+        cids[sidx][tid] = tid >= ncand ? -1
+                          : (pc >= 0 && pc < np) ? pc * QB + tid % QB : -1 - (pc * QB + tid % QB);
       }
-      for (int e = tid; e < (NC + QB) * 16; e += THREADS) {
+#pragma unroll 1
+      for (int e = tid; e < (NC + QB) * 16; e += THREADS) {   // the same trip count in every thread
         const int r = e >> 4, c4 = (e & 15) * 4;
+        const int pc = __shfl_sync(0xffffffffu, pl, (r / QB) & 31);
         if (r < NC) {
-          if (r < ncand) {
-            const int pc = plist[r / QB];
-            if (pc >= 0 && pc < np) cp_async16(&st[sidx].k[r * LD + c4], kbase + ((int64_t)pc * QB + r % QB) * 64 + c4);
-          }
+          if (r < ncand && pc >= 0 && pc < np)
+            cp_async16(&st[sidx].k[r * LD + c4], kbase + ((int64_t)pc * QB + r % QB) * 64 + c4);
         } else {
           cp_async16(&st[sidx].q[(r - NC) * LD + c4], qbase + (r - NC) * 64 + c4);
         }
