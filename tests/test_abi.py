@@ -112,3 +112,25 @@ def test_timeout_selftest_rejects_bad_arguments_before_launch(L):
 def test_status_strings(L):
     for s in range(8):
         assert llsa.status_string(s)
+
+
+@pytest.mark.parametrize("kw, fwd, bwd", [
+    # the metric's workload, and K = all at 256^2 (K_1 = 4096): tensor cores
+    (dict(batch=2, heads=6, height=256, width=256, L=4, K=8), "tensor", "tensor"),
+    (dict(batch=2, heads=6, height=256, width=256, L=1, K=10 ** 6, enrich_mask=0), "tensor", "tensor"),
+    # K = all at 512^2 (K_1 = 16384): above the tensor-core list limit
+    (dict(batch=1, heads=1, height=512, width=512, L=1, K=10 ** 6, enrich_mask=0), "cuda-core", "cuda-core"),
+    # fp32, B = 64 and d = 128 run on the CUDA cores
+    (dict(batch=1, heads=2, height=64, width=64, L=3, K=8, dtype=llsa.FP32), "cuda-core", "cuda-core"),
+    (dict(batch=1, heads=2, height=64, width=64, B=64, L=1, K=8), "cuda-core", "cuda-core"),
+    (dict(batch=1, heads=2, height=64, width=64, d=128, L=3, K=8), "cuda-core", "cuda-core"),
+    # more than 32 pooled keys of levels >= 2 per query block
+    (dict(batch=1, heads=1, height=256, width=256, L=4, K=16), "cuda-core", "cuda-core"),
+])
+def test_attention_dispatch(L, kw, fwd, bwd):
+    """llsa_attn_paths (host only) reports the kernels the problem runs on."""
+    base = dict(d=64, B=16)
+    base.update(kw)
+    p = llsa.Problem(**base)
+    assert llsa.validate(p) == 0
+    assert llsa.attn_paths(p) == {"fwd": fwd, "bwd": bwd}
