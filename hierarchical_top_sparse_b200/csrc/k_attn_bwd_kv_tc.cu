@@ -75,7 +75,9 @@ constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC = 256;
 constexpr int kLast = 1, kFirst = 2;
 enum : int { kEnd = 0, kChunk = 1 };
 // arrivals that free a chunk slot: the MMA thread and each softmax warp
-constexpr int EMPTY_ARRIVALS = 1 + SOFT_WARPS;
+// a chunk slot is freed by both MMA warps (the S / dP warp once it has read the
+// meta words, the dV / dK warp once its MMAs are done) and every softmax warp
+constexpr int EMPTY_ARRIVALS = 2 + SOFT_WARPS;
 constexpr int GRING = 4;            // key-group ids in flight between the producer and the epilogue
 
 struct ChunkSlot {
@@ -380,6 +382,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kv_tc_kernel(
       if (flags & kFirst) ++kseen;
       const int ks = (int)((kseen - 1) & 1);
       if (is_s) {
+        // the meta words are in registers (the tiles are released by the other warp)
+        __syncwarp();
+        if (tc::elect_one()) ptx::mbar_arrive(&s.empty[slot]);
+        __syncwarp();
         if ((flags & kFirst) && !wait(&s.kfull[ks], ((kseen - 1) >> 1) & 1)) break;
         if (nq == 0) continue;
         // the softmax warps have read S / dP of the previous chunk
