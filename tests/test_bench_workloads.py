@@ -56,3 +56,34 @@ def test_sweep_points_are_valid_problems_of_equal_size():
                 assert p.L == 1 and kl[1] == 8 and p.enrich_mask == 1
             else:
                 assert p.L == 1 and kl[1] == n[1] and p.enrich_mask == 0
+
+
+def test_roofline_arithmetic_at_256():
+    """The compulsory bytes and real-pair FLOPs bench.py divides by, at the
+    256 x 256 workload, counted here from the workload itself: 12 slices of
+    65536 tokens, d = 64, B = 16, K = 8, four levels of 4096, 256, 16 and 1
+    tokens, every level enriched."""
+    b = _bench()
+    BH, N, d, L, B = 12, 65536, 64, 4, 16
+    n = [N, 4096, 256, 16, 1]
+    kl = [0, 8, 8, 8, 1]                      # K_4 = min(K, n_4)
+    tok = BH * N * d * 2                      # one bf16 tensor
+    pyr = BH * (4096 + 256 + 16 + 1) * d * 4  # one fp32 pyramid
+    idx = BH * (4096 * 8 + 256 * 8 + 16 * 8 + 1 * 1) * 4
+    offs = BH * (4097 + 257 + 17 + 2) * 4
+    lse = BH * N * 4
+    assert b.algorithmic_bytes("pool", n, kl, BH, N, d, L) == tok + pyr
+    assert b.algorithmic_bytes("select", n, kl, BH, N, d, L) == 2 * pyr + idx
+    assert b.algorithmic_bytes("attn_fwd", n, kl, BH, N, d, L) == 4 * tok + 2 * pyr + idx + lse
+    assert b.algorithmic_bytes("index_transpose", n, kl, BH, N, d, L) == 2 * idx + offs
+    assert b.algorithmic_bytes("attn_bwd", n, kl, BH, N, d, L) == 8 * tok + lse + 2 * pyr + 2 * idx + offs
+    # 128 fine keys and 8 + 8 + 8 + 1 pooled keys per query
+    assert b.keys_per_query(kl, B, L, 0b1111) == 153
+    assert b.keys_per_query(kl, B, L, 0) == 128
+    pairs = BH * N * 153
+    assert b.algorithmic_flops("attn_fwd", kl, BH, N, d, B, L, 0b1111) == pairs * d * 4
+    assert b.algorithmic_flops("attn_bwd", kl, BH, N, d, B, L, 0b1111) == pairs * d * 10
+    # the figures the profiles quote
+    assert round(b.algorithmic_bytes("attn_fwd", n, kl, BH, N, d, L) / 1e6, 1) == 434.3
+    assert round(b.algorithmic_bytes("attn_bwd", n, kl, BH, N, d, L) / 1e6, 1) == 838.9
+    assert round(pairs * d * 4 / 1e9, 1) == 30.8 and round(pairs * d * 10 / 1e9, 1) == 77.0
