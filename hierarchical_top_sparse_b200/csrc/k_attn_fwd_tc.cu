@@ -23,11 +23,11 @@
 // the same for all 256 queries of the token: each group starts with one chunk
 // against them (N = 32, logit bias l ln B).
 //
-// O += P V is issued one key block (16 keys, one K step) at a time, with the
-// rows of the query blocks that did not pick that block disabled in the MMA
-// (tcgen05's per-lane output mask): their accumulators do not change, so the
-// softmax threads write P only for the blocks their rows picked and never
-// write zeros.  The epilogue clears each O buffer after reading it.
+// O += P V is issued one key block (16 keys, one K step) at a time and is not
+// masked: the softmax threads write zero weights for the blocks their rows
+// did not pick.  (tcgen05's per-lane output mask would skip those rows
+// instead, but a masked MMA issues about three times slower than a plain
+// one.)  The epilogue clears each O buffer after reading it.
 //
 // Online softmax with a lazy maximum: a row keeps its running maximum m and
 // rescales O (in TMEM) only when a new logit exceeds m by more than 2^8, so
@@ -570,9 +570,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       const Meta& m = s.meta[ms];
       const int kind = m.kind, nq = m.nq, flags = m.flags;
       const uint32_t gc = (uint32_t)m.gc, tk = (uint32_t)m.tk, kc = (uint32_t)m.kc;
-      int msk[CK];
-#pragma unroll
-      for (int j = 0; j < CK; ++j) msk[j] = m.msk[j];
       __syncwarp();
       if (tc::elect_one()) ptx::mbar_arrive(&s.mempty[ms]);   // the entry is in registers
       __syncwarp();
@@ -783,8 +780,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_tc_kernel(
       }
       if (!wait(&s.p_empty[b], (u & 1) ^ 1, 79)) break;   // the O update of entry sidx - 2 has read P(b)
       tc::fence_after_sync();
-      // P of the blocks this row picked (plus the block's pooled-token share);
-      // the O update skips the rows that did not pick a block
+      // P of the blocks this row picked (plus the block's pooled-token share),
+      // zero for the blocks it did not pick (the O update takes every row)
 #pragma unroll 1
       for (int jj = 0; jj < nblk; ++jj) {
         uint32_t pw[8];
