@@ -15,6 +15,10 @@ ranks of the device time).  Rank 0 prints one JSON line.
 ``--impl reference`` times the CPU oracle (the plain fp64 restatement of the
 method, test infrastructure) on the host cores, on a bounded sample of the
 same workload, and prints the same line with "impl": "reference".
+
+``--workload NAME`` times another forward + backward workload instead, and
+``--sweep`` prints tokens/s against N for LLSA, the single-level top-K
+baseline and dense attention, one JSON line per point.
 """
 from __future__ import annotations
 
