@@ -737,7 +737,7 @@ def cpu_baseline(budget_s: float = 20.0):
         reps += 1
     dt = time.perf_counter() - t
     w = WORKLOAD
-    return {"value": round(tokens / dt, 1), "unit": UNIT, "cores": min(cores, slices * groups), "nproc": cores,
+    return {"value": round(tokens / dt, 1), "unit": UNIT, "cores": slices * groups, "nproc": cores,
             "cpu_model": model, "kind": "oracle",
             "sample": f"{reps} x (pool+select+transpose of {slices} (batch,head) slices of the {w['H']}x{w['W']} "
                       f"workload, attention fwd+bwd for {len(rows)} sampled query rows of each in {groups} "
@@ -766,7 +766,7 @@ def run_reference(args, rank, world, pg):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_desc({"parallelism": "CPU oracle on the host cores (rank 0 only)"}),
-            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": min(cores, slices * groups),
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": slices * groups,
                              "nproc": cores, "cpu_model": model, "kind": "oracle",
                              "sample": f"per step: pool+select+transpose of {slices} (batch,head) slices of the "
                                        f"{WORKLOAD['H']}x{WORKLOAD['W']} workload, attention fwd+bwd for "
